@@ -1,0 +1,383 @@
+"""CPU oracle for the GCA paged KV cache: fp64 NumPy and plain Python.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path imports this module: only the tests,
+the smoke check and the benchmark's CPU-baseline / reference arm do. It shares no code with
+the CUDA library (no kernels, headers, tables or helpers); the only common dependency is the
+seeded input module `gca_inputs`, which holds no method arithmetic.
+
+Sources (web pages, cited by title and section):
+  [GCT]   "How the Geometric Context Transformer Enables Streaming 3D Reconstruction in
+          LingBot-Map" -- sections "Causal Aggregation with KV-Cache Management"
+          (KV-Cache Initialization, 3D Rotary Positional Embeddings), "Attention Blocks:
+          FlashInfer vs. SDPA" (FlashInferBlock), and the FAQ on scale frames / causality.
+  [POOLS] "LingBot-Map runs 10,000 frames on monocular video" -- section "How GCT's
+          Anchor-Pose-Trajectory Pools Make Monocular 3D Tractable".
+  [ABOT]  "Stop hoarding memory: how ABot-Recon reconstructs infinite 3D streams with a fixed
+          12-frame window" -- section "The Local Context Architecture".
+
+What the pages fix: a frame's tokens get 3D (t,y,x) RoPE with t the global frame index
+[GCT, 3D RoPE]; the frame's K/V are appended to a paged cache, frames that left the window are
+evicted, then the frame's queries attend over the cache [GCT, FlashInferBlock]; the cache holds
+three pools -- anchor frame(s), a window of recent frames, and a trajectory pool that keeps a
+few tokens of each evicted frame [POOLS]; attention across frames is causal [GCT, FAQ "Why are
+scale frames processed differently"]; a 12-frame window means 11 cached frames plus the current
+one [ABOT].
+
+Readings where the pages are silent (each is listed in the design notes):
+  R1 token order in a frame: [camera, registers, patches row-major over (grid_h, grid_w)].
+  R2 RoPE band split d_y = d_x = 2*floor(D/6), d_t = D - d_y - d_x, order (t, y, x);
+     interleaved pairs (2j, 2j+1); pair j of a band of width d turns by pos * base**(-2j/d);
+     a patch at (row r, col c) sits at (t, r+1, c+1), special tokens at (t, 0, 0); q and k
+     rotate, v does not; k is cached rotated.
+  R3 pools at step t, in order append -> evict -> attend: anchor = frames 0..A-1;
+     window = frames max(A, t-W+1)..t (W counts the current frame); trajectory = kept tokens
+     of frames A..t-W. Before frame A the frame sees frames 0..t. No mask inside a frame.
+  R4 kept tokens: K <= S -> tokens 0..K-1; else all S special tokens plus patches
+     S + j*floor(P/(K-S)), j = 0..K-S-1. Trajectory order: by evicted frame, then kept index.
+  R5 softmax scale 1/sqrt(D).
+  R6 allocator: FIFO free list. Append pops ceil(T/ps) pages for the frame (frames start
+     page-aligned); eviction then copies the kept tokens to the trajectory tail, popping a
+     page whenever the tail page is full (trajectory pages are dense and never freed), and
+     finally pushes the evicted frame's pages to the tail in row order. Anchor pages are
+     never freed. Reset restores the initial order.
+"""
+from __future__ import annotations
+
+import math
+from collections import deque
+
+import numpy as np
+
+__all__ = [
+    "OutOfPages",
+    "rope_band_widths",
+    "token_positions",
+    "rope_angles",
+    "rotate_pairs",
+    "kept_token_indices",
+    "pool_frames",
+    "visible_keys",
+    "visible_key_count",
+    "softmax_attention",
+    "FifoPages",
+    "CacheBook",
+    "GcaOracle",
+]
+
+
+class OutOfPages(RuntimeError):
+    pass
+
+
+# --------------------------------------------------------------------------------------
+# 3D RoPE [GCT, "3D Rotary Positional Embeddings"; reading R2]
+# --------------------------------------------------------------------------------------
+
+def rope_band_widths(head_dim: int):
+    """(d_t, d_y, d_x): two spatial bands of 2*floor(D/6) dims each, the rest for time."""
+    d_sp = 2 * (head_dim // 6)
+    return head_dim - 2 * d_sp, d_sp, d_sp
+
+
+def token_positions(t: int, num_special: int, grid_h: int, grid_w: int) -> np.ndarray:
+    """int64 [T, 3] positions (t, y, x) of frame t's tokens, token order R1."""
+    T = num_special + grid_h * grid_w
+    pos = np.zeros((T, 3), dtype=np.int64)
+    pos[:, 0] = t
+    for p in range(grid_h * grid_w):
+        r, c = divmod(p, grid_w)
+        pos[num_special + p, 1] = r + 1
+        pos[num_special + p, 2] = c + 1
+    return pos
+
+
+def rope_angles(pos: np.ndarray, head_dim: int, base: float) -> np.ndarray:
+    """fp64 [N, D/2] rotation angle of every pair: band b of width d gives pair j the
+    angle pos_b * base**(-2j/d)."""
+    widths = rope_band_widths(head_dim)
+    cols = []
+    for b, d in enumerate(widths):
+        j = np.arange(d // 2, dtype=np.float64)
+        inv_freq = np.power(float(base), -2.0 * j / d)
+        cols.append(pos[:, b : b + 1].astype(np.float64) * inv_freq[None, :])
+    return np.concatenate(cols, axis=1)
+
+
+def rotate_pairs(x: np.ndarray, angles: np.ndarray) -> np.ndarray:
+    """Rotate interleaved pairs (x[2j], x[2j+1]) by angles[..., j].
+
+    x: fp64 [N, H, D]; angles: [N, D/2]. Returns fp64 [N, H, D].
+    """
+    a = x[..., 0::2]
+    b = x[..., 1::2]
+    c = np.cos(angles)[:, None, :]
+    s = np.sin(angles)[:, None, :]
+    out = np.empty_like(x)
+    out[..., 0::2] = a * c - b * s
+    out[..., 1::2] = a * s + b * c
+    return out
+
+
+# --------------------------------------------------------------------------------------
+# Pools [POOLS; GCT FlashInferBlock order append -> evict -> attend; readings R3, R4]
+# --------------------------------------------------------------------------------------
+
+def kept_token_indices(num_special: int, num_patches: int, keep: int):
+    """Token indices an evicted frame keeps in the trajectory pool (reading R4)."""
+    if keep <= 0:
+        return []
+    if keep <= num_special:
+        return list(range(keep))
+    extra = keep - num_special
+    stride = num_patches // extra
+    if stride < 1:
+        raise ValueError("more kept patches than patches")
+    return list(range(num_special)) + [num_special + j * stride for j in range(extra)]
+
+
+def pool_frames(t: int, A: int, W: int):
+    """(anchor frames, window frames, evicted frames) visible at step t (reading R3)."""
+    if t < A:
+        return list(range(t + 1)), [], []
+    anchor = list(range(A))
+    w0 = max(A, t - W + 1)
+    window = list(range(w0, t + 1))
+    evicted = list(range(A, w0))
+    return anchor, window, evicted
+
+
+def visible_keys(t: int, A: int, W: int, T: int, kept):
+    """Pool-ordered list of (frame, token) keys that frame t's queries see."""
+    anchor, window, evicted = pool_frames(t, A, W)
+    keys = [(f, i) for f in anchor for i in range(T)]
+    keys += [(f, i) for f in window for i in range(T)]
+    keys += [(f, i) for f in evicted for i in kept]
+    return keys
+
+
+def visible_key_count(t: int, A: int, W: int, T: int, K: int) -> int:
+    anchor, window, evicted = pool_frames(t, A, W)
+    return (len(anchor) + len(window)) * T + len(evicted) * K
+
+
+# --------------------------------------------------------------------------------------
+# Attention: softmax(q k^T / sqrt(D)) v over the visible keys [GCT compute_attention; R5]
+# --------------------------------------------------------------------------------------
+
+def softmax_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
+    """fp64 attention of one head. q [Nq, D], k [Nk, D], v [Nk, D] -> [Nq, D]."""
+    d = q.shape[-1]
+    s = (q @ k.T) / math.sqrt(d)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    return (p @ v) / p.sum(axis=1, keepdims=True)
+
+
+# --------------------------------------------------------------------------------------
+# Page bookkeeping [GCT "paged KV cache", KV-Cache Initialization; reading R6]
+# --------------------------------------------------------------------------------------
+
+class FifoPages:
+    """FIFO free list of physical page ids."""
+
+    def __init__(self, initial_order):
+        self.initial = [int(p) for p in initial_order]
+        self.free = deque(self.initial)
+
+    def pop(self) -> int:
+        if not self.free:
+            raise OutOfPages("free list empty")
+        return self.free.popleft()
+
+    def push(self, page: int) -> None:
+        self.free.append(page)
+
+    def reset(self) -> None:
+        self.free = deque(self.initial)
+
+
+class CacheBook:
+    """Integer state of one cache: page rows per frame, slot map, trajectory pages.
+
+    Spells out the allocator reading R6 step by step; every GPU page id is compared with it.
+    """
+
+    def __init__(self, *, T, page_size, anchor_frames, window_frames, kept, initial_free):
+        self.T = T
+        self.ps = page_size
+        self.A = anchor_frames
+        self.W = window_frames
+        self.kept = list(kept)
+        self.ppf = -(-T // page_size)
+        self.alloc = FifoPages(initial_free)
+        self.reset()
+
+    def reset(self):
+        self.alloc.reset()
+        self.frame_pages = {}  # frame -> list of page ids (live frames)
+        self.all_rows = {}  # frame -> page row (also kept after eviction, for inspection)
+        self.traj_pages = []
+        self.traj_tokens = []  # (frame, token) per trajectory slot, in order
+        self.frames = 0
+        self.slot_map = []
+
+    @property
+    def traj_len(self):
+        return len(self.traj_tokens)
+
+    def pages_in_use(self):
+        return sum(len(r) for r in self.frame_pages.values()) + len(self.traj_pages)
+
+    def append(self, t: int):
+        if t != self.frames:
+            raise ValueError("frames must be appended in order")
+        # 1. the new frame's pages, popped in order
+        row = [self.alloc.pop() for _ in range(self.ppf)]
+        self.frame_pages[t] = row
+        self.all_rows[t] = row
+        self.slot_map = [row[i // self.ps] * self.ps + i % self.ps for i in range(self.T)]
+        # 2. eviction of the frame that left the window
+        e = t - self.W
+        if e >= self.A:
+            for i in self.kept:
+                if self.traj_len % self.ps == 0:
+                    self.traj_pages.append(self.alloc.pop())
+                self.traj_tokens.append((e, i))
+            for p in self.frame_pages.pop(e):
+                self.alloc.push(p)
+        self.frames += 1
+
+    def location_of(self, frame: int, token: int):
+        """(page, slot) that holds a live frame's token."""
+        row = self.frame_pages[frame]
+        return row[token // self.ps], token % self.ps
+
+    def traj_location(self, n: int):
+        return self.traj_pages[n // self.ps], n % self.ps
+
+
+# --------------------------------------------------------------------------------------
+# Whole stream
+# --------------------------------------------------------------------------------------
+
+class GcaOracle:
+    """fp64 oracle of one GCA cache fed by a seeded synthetic stream.
+
+    `frame_source(t)` returns the bf16 (q, k, v) tensors [T, H, D] of frame t (torch or
+    numpy); they are widened exactly. `slot_of(t)` names the distinct input frame that frame t
+    reuses (identity by default), so long streams keep a bounded set of raw frames in memory.
+    """
+
+    def __init__(self, *, num_heads, head_dim, page_size, grid_h, grid_w, num_special,
+                 anchor_frames, window_frames, keep_tokens, rope_base, initial_free,
+                 frame_source, slot_of=None):
+        self.H = num_heads
+        self.D = head_dim
+        self.ps = page_size
+        self.gh = grid_h
+        self.gw = grid_w
+        self.S = num_special
+        self.P = grid_h * grid_w
+        self.T = self.S + self.P
+        self.A = anchor_frames
+        self.W = window_frames
+        self.K = keep_tokens
+        self.base = rope_base
+        self.kept = kept_token_indices(self.S, self.P, self.K)
+        self.source = frame_source
+        self.slot_of = slot_of if slot_of is not None else (lambda t: t)
+        self.book = CacheBook(T=self.T, page_size=page_size, anchor_frames=anchor_frames,
+                              window_frames=window_frames, kept=self.kept,
+                              initial_free=initial_free)
+        self._raw = {}  # slot -> (q, k, v) as float32 arrays (exact copies of bf16)
+        self._pos = token_positions(0, self.S, self.gh, self.gw)
+
+    # inputs ---------------------------------------------------------------------------
+    def raw32(self, t):
+        slot = self.slot_of(t)
+        if slot not in self._raw:
+            q, k, v = self.source(t)
+            self._raw[slot] = tuple(_to_f32(x) for x in (q, k, v))
+        return self._raw[slot]
+
+    def raw(self, t):
+        return tuple(x.astype(np.float64) for x in self.raw32(t))
+
+    def positions(self, frames, tokens):
+        """int64 [N, 3] positions of the (frame, token) pairs."""
+        frames = np.asarray(frames, dtype=np.int64)
+        tokens = np.asarray(tokens, dtype=np.int64)
+        pos = self._pos[tokens].copy()
+        pos[:, 0] = frames
+        return pos
+
+    def q_rot(self, t, rows=None):
+        toks = np.arange(self.T) if rows is None else np.asarray(rows)
+        q = self.raw32(t)[0][toks].astype(np.float64)
+        ang = rope_angles(self.positions(np.full(len(toks), t), toks), self.D, self.base)
+        return rotate_pairs(q, ang)
+
+    def k_rot(self, t, tokens=None):
+        toks = np.arange(self.T) if tokens is None else np.asarray(tokens)
+        k = self.raw32(t)[1][toks].astype(np.float64)
+        ang = rope_angles(self.positions(np.full(len(toks), t), toks), self.D, self.base)
+        return rotate_pairs(k, ang)
+
+    # bookkeeping ----------------------------------------------------------------------
+    def append(self, t):
+        self.book.append(t)
+
+    def visible(self, t):
+        return visible_keys(t, self.A, self.W, self.T, self.kept)
+
+    def key_index(self, t):
+        """(frames, tokens) int arrays of the keys frame t sees, in pool order."""
+        anchor, window, evicted = pool_frames(t, self.A, self.W)
+        full = np.asarray(anchor + window, dtype=np.int64)
+        fr = [np.repeat(full, self.T)]
+        tk = [np.tile(np.arange(self.T, dtype=np.int64), len(full))]
+        if evicted and self.kept:
+            ev = np.asarray(evicted, dtype=np.int64)
+            fr.append(np.repeat(ev, len(self.kept)))
+            tk.append(np.tile(np.asarray(self.kept, dtype=np.int64), len(ev)))
+        return np.concatenate(fr), np.concatenate(tk)
+
+    def gather_head(self, t, h, frames=None, tokens=None, angles=None):
+        """fp64 (K_rot, V) [Nk, D] of head h over the keys frame t sees, in pool order."""
+        if frames is None:
+            frames, tokens = self.key_index(t)
+        if angles is None:
+            angles = rope_angles(self.positions(frames, tokens), self.D, self.base)
+        k = np.empty((len(frames), self.D), dtype=np.float64)
+        v = np.empty((len(frames), self.D), dtype=np.float64)
+        slots = np.asarray([self.slot_of(int(f)) for f in frames])
+        for s in np.unique(slots):
+            sel = np.nonzero(slots == s)[0]
+            f0 = int(frames[sel[0]])
+            _, kr, vr = self.raw32(f0)
+            k[sel] = kr[tokens[sel], h, :]
+            v[sel] = vr[tokens[sel], h, :]
+        k = rotate_pairs(k[:, None, :], angles)[:, 0, :]
+        return k, v
+
+    def attend(self, t, rows=None):
+        """fp64 attention output [len(rows), H, D] of frame t's query rows."""
+        qr = self.q_rot(t, rows)
+        frames, tokens = self.key_index(t)
+        angles = rope_angles(self.positions(frames, tokens), self.D, self.base)
+        out = np.empty_like(qr)
+        for h in range(self.H):
+            k, v = self.gather_head(t, h, frames, tokens, angles)
+            out[:, h, :] = softmax_attention(qr[:, h, :], k, v)
+        return out
+
+
+def _to_f32(x):
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            return x.to(torch.float32).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x, dtype=np.float32)
