@@ -1,0 +1,498 @@
+"""Benchmark of the GCA paged KV cache hot path on B200.
+
+One step = one whole stream of the 320-frame workload through one cache: gca_reset, then for
+every frame t: gca_append_frame (RoPE + paged append + eviction) and gca_attend (three-pool
+paged attention, split-KV combine). Inputs come from a device-resident ring of 64 distinct
+frames (395 MB, larger than the 126 MB L2). Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank streams its own replica (no collective on the data path; weak
+scaling); the timed region is bracketed by a barrier and synchronisation and its duration is
+the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gca_inputs as gi  # noqa: E402
+
+METRIC = "GCA frames/sec and attention TFLOP/s (% of BF16 peak) at 1 B200"
+WORKLOAD = "w16_320"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def workload_desc(w: gi.Workload) -> str:
+    return (f"one GCA layer at 518x378: {w.tokens_per_frame} tokens/frame "
+            f"({w.grid_h}x{w.grid_w} patches + {w.num_special} special), {w.num_heads} heads x "
+            f"{w.head_dim}, page 16, anchor {w.anchor_frames}, window {w.window_frames}, "
+            f"{w.keep_tokens} kept tokens per evicted frame, {w.frames}-frame stream")
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def visible_keys(w: gi.Workload, t: int) -> int:
+    """Nk(t) as the cache reports it is preferred; this is only for the CPU-baseline estimate."""
+    A, W, T, K = w.anchor_frames, w.window_frames, w.tokens_per_frame, w.keep_tokens
+    if t < A:
+        return (t + 1) * T
+    return A * T + min(W, t + 1 - A) * T + max(0, t + 1 - A - W) * K
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, out_path: str | None):
+        self.index = index
+        self.proc = None
+        self.path = out_path
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w") if self.path else subprocess.PIPE
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.text = ""
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        if self.path:
+            self.f.close()
+            out = open(self.path).read()
+        self.text = out or ""
+
+    def summary(self):
+        rows = []
+        for line in getattr(self, "text", "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9], parts[4]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [r[0] for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Maximum of a per-rank duration over all ranks (all_reduce MAX); identity at world 1."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_frames_per_s(world: int, steps: int, frames: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank streams `steps` replicas of `frames` frames."""
+    return world * steps * frames / (max_ms / 1e3)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("gca_attn.cu", "gca_append.cu", "gca_internal.h"):
+        h.update(open(os.path.join(ROOT, "paged_kv_cache_gca_b200", "csrc", name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernels."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    ent = d.get(kernel)
+    if not ent or ent.get("source_hash") != kernel_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def run_ours(args, rank, world, device):
+    import paged_kv_cache_gca_b200 as gca
+    from paged_kv_cache_gca_b200 import build as gbuild
+
+    gbuild.build()
+    w = gi.workload(args.workload)
+    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    stream = torch.cuda.Stream(device=device)
+    ring_host = gi.draw_ring(w)  # [R, 3, T, H, D] bf16, CPU
+    ring = ring_host.to(device)
+    with torch.cuda.stream(stream):
+        cache = gca.GcaCache(gca.config_for(w), initial_free=gi.initial_free_list(w),
+                             stream=stream)
+    q_rot = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
+    out = torch.empty_like(q_rot)
+    nframes = w.frames
+
+    # per-frame work (host values the library reports)
+    flops = []
+    info_launches = []
+
+    def one_step(events=None):
+        cache.reset(stream=stream)
+        for t in range(nframes):
+            q, k, v = ring[t % w.ring]
+            if events is not None:
+                events[t][0].record(stream)
+            cache.append_frame(t, q, k, v, q_rot, stream=stream)
+            if events is not None:
+                events[t][1].record(stream)
+            cache.attend(t, q_rot, out, stream=stream)
+            if events is not None:
+                events[t][2].record(stream)
+            if len(flops) < nframes:
+                inf = cache.attend_info()
+                flops.append(4.0 * H * D * T * inf.visible_keys)
+                info_launches.append(inf.launches)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one_step()
+    torch.cuda.synchronize(device)
+    assert cache.check() == 0, "device error after warm-up"
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # one event triple per (step, frame): read only after the timed region
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nframes)]
+          for _ in range(args.steps)]
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_stop = torch.cuda.Event(enable_timing=True)
+    clocks_path = os.path.join(ROOT, "gpurun_out", "bench_clocks.csv") if os.path.isdir(
+        os.path.join(ROOT, "gpurun_out")) else None
+    with ClockSampler(torch.cuda.current_device() if device.index is None else device.index,
+                      clocks_path if rank == 0 else None) as clk:
+        barrier()
+        torch.cuda.synchronize(device)
+        e_start.record(stream)
+        with torch.cuda.stream(stream):
+            for s in range(args.steps):
+                one_step(ev[s])
+        e_stop.record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+    append_ms = sum(e[0].elapsed_time(e[1]) for st in ev for e in st)
+    attend_ms = sum(e[1].elapsed_time(e[2]) for st in ev for e in st)
+    elapsed_ms = e_start.elapsed_time(e_stop)
+    assert cache.check() == 0, "device error in the timed region"
+    step_ms_calls = (append_ms + attend_ms) / args.steps
+
+    elapsed_ms = max_over_ranks(elapsed_ms, world, device)
+
+    # ---- end-to-end through the public API with host buffers (pinned), copies timed
+    e2e = run_e2e(args, w, cache, ring_host, device, stream, world)
+
+    res = {
+        "elapsed_ms": elapsed_ms,
+        "step_ms_calls": step_ms_calls,
+        "attend_ms_per_step": attend_ms / args.steps,
+        "append_ms_per_step": append_ms / args.steps,
+        "flops_per_step": float(sum(flops)),
+        "launches_per_step": 1 + nframes + int(sum(info_launches)),
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "frames": nframes,
+    }
+    cache.close()
+    return w, res
+
+
+def run_e2e(args, w, cache, ring_host, device, stream, world):
+    """Frames/s through the public API with inputs in pinned host memory: every frame's q, k, v
+    are copied host->device and its output device->host inside the timed region. Copies run on
+    a second stream so frame t+1's upload overlaps frame t's compute."""
+    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    pinned = ring_host.pin_memory()
+    out_host = torch.empty((2, T, H, D), dtype=torch.bfloat16).pin_memory()
+    inp = [torch.empty((3, T, H, D), dtype=torch.bfloat16, device=device) for _ in range(2)]
+    q_rot = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
+    out = [torch.empty((T, H, D), dtype=torch.bfloat16, device=device) for _ in range(2)]
+    copy = torch.cuda.Stream(device=device)
+    up = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    nframes = w.frames
+    steps = max(1, min(args.steps, 3))
+
+    def step():
+        cache.reset(stream=stream)
+        with torch.cuda.stream(copy):
+            inp[0].copy_(pinned[0], non_blocking=True)
+            up[0].record(copy)
+        for t in range(nframes):
+            b = t & 1
+            if t + 1 < nframes:
+                nb = (t + 1) & 1
+                with torch.cuda.stream(copy):
+                    if t >= 1:
+                        copy.wait_event(done[nb])  # buffer nb was last used by frame t-1
+                    inp[nb].copy_(pinned[(t + 1) % w.ring], non_blocking=True)
+                    up[nb].record(copy)
+            stream.wait_event(up[b])
+            cache.append_frame(t, inp[b][0], inp[b][1], inp[b][2], q_rot, stream=stream)
+            cache.attend(t, q_rot, out[b], stream=stream)
+            with torch.cuda.stream(stream):
+                out_host[b].copy_(out[b], non_blocking=True)
+            done[b].record(stream)
+
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    copy.synchronize()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    frame_bytes = T * H * D * 2
+    return {"value": aggregate_frames_per_s(world, steps, nframes, ms), "unit": "frames/s",
+            "h2d_bytes_per_step": 3 * frame_bytes * nframes,
+            "d2h_bytes_per_step": frame_bytes * nframes, "steps": steps}
+
+
+# ----------------------------------------------------------------------------- oracle
+
+def oracle_sample(w: gi.Workload, frames_to_attend, rows=None):
+    """Runs the CPU oracle: bookkeeping over the stream up to the last sampled frame, attention
+    on the sampled frames. Returns (seconds bookkeeping, seconds attention, frames)."""
+    import oracle as orc
+
+    o = orc.GcaOracle(num_heads=w.num_heads, head_dim=w.head_dim, page_size=w.page_size,
+                      grid_h=w.grid_h, grid_w=w.grid_w, num_special=w.num_special,
+                      anchor_frames=w.anchor_frames, window_frames=w.window_frames,
+                      keep_tokens=w.keep_tokens, rope_base=w.rope_base,
+                      initial_free=gi.initial_free_list(w).tolist(),
+                      frame_source=lambda t: gi.draw_frame(w, t),
+                      slot_of=lambda t: t % w.ring)
+    for s in range(w.ring):  # inputs drawn before the clock starts
+        o.raw32(s)
+    t_book = t_att = 0.0
+    todo = sorted(frames_to_attend)
+    for t in range(w.frames):
+        a = time.perf_counter()
+        o.append(t)
+        t_book += time.perf_counter() - a
+        if todo and t == todo[0]:
+            todo.pop(0)
+            a = time.perf_counter()
+            o.attend(t, rows)
+            t_att += time.perf_counter() - a
+    return t_book, t_att
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return torch.get_num_threads()
+
+
+def oracle_frames_per_s(w: gi.Workload, sample_frames):
+    """Oracle frames/s on this host, extrapolated from a bounded sample: bookkeeping is timed
+    over the whole stream; attention on the sampled frames (all rows, all heads) gives a cost
+    per query-key pair that is applied to every frame's T x Nk(t)."""
+    t_book, t_att = oracle_sample(w, sample_frames)
+    T = w.tokens_per_frame
+    sampled_pairs = sum(T * visible_keys(w, t) for t in sample_frames)
+    all_pairs = sum(T * visible_keys(w, t) for t in range(w.frames))
+    est = t_book + t_att * all_pairs / sampled_pairs
+    return w.frames / est, {
+        "bookkeeping_s": round(t_book, 3), "attention_s_sampled": round(t_att, 3),
+        "estimated_stream_s": round(est, 3)}
+
+
+def run_reference(args):
+    w = gi.workload(args.workload)
+    rng = np.random.default_rng(12345)
+    values, details = [], []
+    per_step = 2
+    t0 = time.perf_counter()
+    for s in range(args.warmup + args.steps):
+        frames = sorted(int(x) for x in rng.choice(w.frames, per_step, replace=False))
+        v, d = oracle_frames_per_s(w, frames)
+        if s >= args.warmup:
+            values.append(v)
+            details.append({"frames": frames, **d})
+    wall = time.perf_counter() - t0
+    value = float(np.mean(values))
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "frames/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * w.frames / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: " + workload_desc(w), "frames_per_step": w.frames},
+        "cpu_baseline": {"value": value, "unit": "frames/s", "cores": cores, "kind": "oracle",
+                         "sample": (f"per step: FIFO bookkeeping over all {w.frames} frames + "
+                                    f"fp64 attention (all rows, heads) of {per_step} random "
+                                    "frames, extrapolated to the stream by query-key pairs")},
+        "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": round(wall, 1), "steps_detail": details[:3],
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        sys.exit(1)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    w, r = run_ours(args, rank, world, device)
+    pk, pk_kind = peaks()
+    value = aggregate_frames_per_s(world, args.steps, r["frames"], r["elapsed_ms"])
+    att_tflops = r["flops_per_step"] / (r["attend_ms_per_step"] / 1e3) / 1e12
+    peak_t = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    att_traffic = traffic_from_profile("attn")
+    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    append_bytes = 6.0 * T * H * D * 2
+    evict_bytes = 4.0 * w.keep_tokens * H * D * 2
+    evictions = max(0, w.frames - w.anchor_frames - w.window_frames)
+    app_bytes_step = append_bytes * w.frames + evict_bytes * evictions
+    app_gbs = app_bytes_step / (r["append_ms_per_step"] / 1e3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "frames/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": r["elapsed_ms"] / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{w.name}: " + workload_desc(w),
+            "frames_per_step": w.frames,
+            "step": "gca_reset + per frame gca_append_frame + gca_attend",
+            "l2": "inputs larger than L2: 64-frame q/k/v ring (395 MB) on the device",
+            "parallelism": "replicas" if world > 1 else "single GPU",
+        },
+        "attention_tflops": att_tflops,
+        "attention_frac_of_bf16_peak": att_tflops / peak_t,
+        "roofline": {
+            "kernel": "gca_attend (tcgen05 paged attention + split-KV combine)",
+            "bound": "tensor", "achieved": att_tflops, "peak": peak_t, "unit": "TFLOP/s",
+            "frac": att_tflops / peak_t,
+            "peak_kind": f"bf16 sustained, {pk_kind}",
+            "frac_of_burst_peak": att_tflops / pk["bf16_tflops"],
+            "traffic": att_traffic,
+            "flops_per_step": r["flops_per_step"],
+        },
+        "append_roofline": {
+            "kernel": "gca_append_frame (RoPE + paged scatter + eviction)",
+            "bound": "hbm", "achieved": app_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": app_gbs / pk["hbm_gbs"], "peak_kind": pk_kind,
+            "bytes_per_step": app_bytes_step,
+            "us_per_append": 1e3 * r["append_ms_per_step"] / w.frames,
+        },
+        "e2e": r["e2e"],
+        "gpu_launches": r["launches_per_step"] * args.steps,
+        "clocks": r["clocks"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, d = oracle_frames_per_s(w, [w.frames // 2, w.frames - 1])
+        line["cpu_baseline"] = {
+            "value": v, "unit": "frames/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"FIFO bookkeeping over all {w.frames} frames + fp64 attention (all rows "
+                       f"and heads) of frames {w.frames // 2} and {w.frames - 1}, extrapolated "
+                       "to the stream by query-key pairs"),
+            **d,
+        }
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+/*
+ * gca.h -- C ABI of the B200 (sm_100a) paged KV cache for Geometric Context Attention.
+ *
+ * One cache serves one attention layer of a streaming video transformer. Every frame:
+ *   1. its tokens' q and k get 3D (t, y, x) rotary embeddings, t being the global frame index
+ *      ("How the Geometric Context Transformer Enables Streaming 3D Reconstruction in
+ *      LingBot-Map", section "3D Rotary Positional Embeddings");
+ *   2. its k (rotated) and v are appended to device pages; the frame that left the sliding
+ *      window is evicted, keeping only a few tokens in the trajectory pool
+ *      (same page, section "FlashInferBlock": append_frame, then evict_frames);
+ *   3. its queries attend with an online softmax over three pools -- anchor frame(s), the window
+ *      of recent frames and the trajectory pool ("LingBot-Map runs 10,000 frames on monocular
+ *      video", section "How GCT's Anchor-Pose-Trajectory Pools Make Monocular 3D Tractable";
+ *      FlashInferBlock: compute_attention).
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *   - token order in a frame: camera, registers, then patches row-major over (grid_h, grid_w);
+ *   - RoPE: bands d_y = d_x = 2*floor(D/6), d_t = D - d_y - d_x in the order (t, y, x);
+ *     interleaved pairs (2j, 2j+1); pair j of a band of width d turns by pos * base^(-2j/d);
+ *     a patch at row r, column c is at (t, r+1, c+1); camera/register tokens at (t, 0, 0);
+ *   - window W counts the current frame; at frame t the window is frames max(A, t-W+1)..t and
+ *     frame t-W (if >= A) is evicted; anchors (frames 0..A-1) are never evicted;
+ *   - kept tokens of an evicted frame: K <= S: tokens 0..K-1; otherwise all S special tokens
+ *     plus patches S + j*floor(P/(K-S)), j = 0..K-S-1;
+ *   - attention scale 1/sqrt(D); no mask inside the current frame; frame-causal across frames;
+ *   - pages: FIFO free list; a frame takes ceil(T/page_size) pages (page-aligned); the
+ *     trajectory pool is dense (page_size tokens per page) and never freed; the evicted
+ *     frame's pages go back to the tail of the free list in row order.
+ *
+ * Tensors are raw device pointers, bf16, contiguous, token-major "NHD": [T][H][D].
+ * Streams are cudaStream_t passed as void* (NULL = legacy default stream).
+ * Calls that enqueue work never synchronise; only gca_check() does.
+ * Supported sizes: head_dim 64, page_size 16, 1 <= num_heads <= 64, keep_tokens <= 64.
+ */
+#ifndef GCA_H_
+#define GCA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct gca_cache gca_cache; /* opaque host handle */
+
+typedef enum {
+  GCA_OK = 0,
+  GCA_ERR_INVALID_ARG = -1,  /* bad pointer, size or config value */
+  GCA_ERR_OUT_OF_PAGES = -2, /* the step needs more free pages than the pool has */
+  GCA_ERR_FRAME_ORDER = -3,  /* frame_idx is not the next frame (append) / last frame (attend) */
+  GCA_ERR_CUDA = -4,         /* a CUDA runtime call failed */
+  GCA_ERR_UNSUPPORTED = -5,  /* valid but not implemented size (e.g. head_dim != 64) */
+  GCA_ERR_DEVICE = -6        /* a kernel set the cache's sticky device error word */
+} gca_status;
+
+/* Device error bits (gca_state.device_error after gca_check). */
+#define GCA_DEVERR_PAGE_RANGE 0x1u   /* a page id read from device state was out of range */
+#define GCA_DEVERR_WAIT_TIMEOUT 0x2u /* a pipeline wait in the attention kernel gave up */
+#define GCA_DEVERR_FREE_LIST 0x4u    /* the initial free list is not a permutation */
+#define GCA_DEVERR_SMEM_ALIGN 0x8u   /* attention kernel: shared memory base not 1024-aligned */
+
+typedef struct {
+  int32_t num_heads;     /* H */
+  int32_t head_dim;      /* D; 64 */
+  int32_t page_size;     /* tokens per page; 16 */
+  int32_t grid_h;        /* patch rows per frame */
+  int32_t grid_w;        /* patch columns per frame */
+  int32_t num_special;   /* S: camera + register tokens; T = S + grid_h * grid_w */
+  int32_t anchor_frames; /* A >= 0 */
+  int32_t window_frames; /* W >= 1, counts the current frame */
+  int32_t keep_tokens;   /* K >= 0 tokens kept per evicted frame (0: no trajectory pool) */
+  int32_t max_frames;    /* frames one stream may append before gca_reset (RoPE table length) */
+  int32_t num_pages;     /* physical page capacity of the pool */
+  float rope_base;       /* RoPE theta (> 1) */
+} gca_config;
+
+/* Host-mirrored counters and device addresses of a cache's state. Filling it never touches the
+ * GPU. All device arrays live inside the caller's workspace. */
+typedef struct {
+  int64_t frames_appended;
+  int64_t free_head;    /* the free list is ring[(free_head .. free_tail-1) mod num_pages] */
+  int64_t free_tail;
+  int64_t traj_len;     /* tokens in the trajectory pool */
+  int32_t traj_pages;   /* pages held by the trajectory pool */
+  int32_t tokens_per_frame;
+  int32_t pages_per_frame;
+  int32_t pages_in_use;
+  uint32_t device_error; /* last value read by gca_check() */
+  int32_t reserved;
+  void* k_pool;          /* bf16 [num_pages][H][page_size][D]: rotated keys */
+  void* v_pool;          /* bf16 [num_pages][H][page_size][D]: values */
+  int32_t* free_ring;    /* int32 [num_pages] */
+  int32_t* frame_pages;  /* int32 [max_frames][pages_per_frame]: page row of every frame */
+  int32_t* traj_page_list; /* int32 [trajectory page capacity] */
+  int32_t* slot_map;     /* int32 [T]: page*page_size + slot of the last appended frame's tokens */
+  int32_t* kept_tokens;  /* int32 [K]: token indices an evicted frame keeps */
+} gca_state;
+
+/* Work description of the last gca_attend() call (host values, for measurement). */
+typedef struct {
+  int64_t frame_idx;
+  int64_t visible_keys;  /* Nk(t): keys the frame's queries see */
+  int32_t logical_pages; /* pages walked, incl. partially filled ones */
+  int32_t kv_tiles;      /* 128-key tiles per query tile */
+  int32_t query_tiles;   /* 128-query tiles per head */
+  int32_t grid;          /* CTAs of the attention kernel */
+  int32_t split;         /* 1 if any (head, query tile) was split across CTAs (combine ran) */
+  int32_t launches;      /* kernels enqueued by the call */
+} gca_attend_info;
+
+/* Validates a config. Host only. Returns GCA_OK, GCA_ERR_INVALID_ARG or GCA_ERR_UNSUPPORTED. */
+gca_status gca_validate_config(const gca_config* cfg);
+
+/* Bytes of device workspace a cache with this config needs (0 if the config is invalid).
+ * Host only; the size does not depend on the GPU. */
+size_t gca_workspace_bytes(const gca_config* cfg);
+
+/* Creates a cache inside a caller-owned device workspace (>= gca_workspace_bytes, 1024-byte
+ * aligned). Enqueues initialisation on `stream` (zeroed pools, RoPE tables, free list).
+ * dev_initial_free_list: NULL for the order 0..num_pages-1, else a device array int32
+ * [num_pages] holding a permutation (the free list's initial order; copied, and restored by
+ * gca_reset). A non-permutation sets GCA_DEVERR_FREE_LIST, reported by gca_check.
+ * The workspace must stay allocated until gca_cache_destroy. Ownership: the caller owns the
+ * workspace; the library owns only *out. The GPU current at this call is the cache's device. */
+gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t ws_bytes,
+                            const int32_t* dev_initial_free_list, void* stream,
+                            gca_cache** out);
+
+/* Appends frame `frame_idx` (pages' append_frame, then evict_frames):
+ * RoPE on q and k, k_rot and v scattered into freshly popped pages, q_rot written for
+ * gca_attend, and the frame that leaves the window evicted (kept tokens copied to the
+ * trajectory tail, its pages pushed back to the free list) -- one kernel launch.
+ * q, k, v: device bf16 [T][H][D]; q_rot_out: device bf16 [T][H][D] (may alias q).
+ * frame_idx must equal the number of frames appended since create/reset
+ * (GCA_ERR_FRAME_ORDER) and be < max_frames. The page budget is checked on the host from
+ * mirrored counts: GCA_ERR_OUT_OF_PAGES returns with nothing enqueued. */
+gca_status gca_append_frame(gca_cache* cache, int64_t frame_idx, const void* q, const void* k,
+                            const void* v, void* q_rot_out, void* stream);
+
+/* Attention of the last appended frame's queries over the cache (pages' compute_attention):
+ * out[i][h] = softmax_j(q_rot[i][h] . k_j[h] / sqrt(D)) v_j[h] over the anchor, window and
+ * trajectory keys visible at frame frame_idx (which must be the last appended frame).
+ * q_rot: device bf16 [T][H][D] from gca_append_frame; out: device bf16 [T][H][D].
+ * One tcgen05 attention launch, plus one combine launch when the key range is split. */
+gca_status gca_attend(gca_cache* cache, int64_t frame_idx, const void* q_rot, void* out,
+                      void* stream);
+
+/* Restores the state of a new stream (pages' clean_kv_cache): free list back to its initial
+ * order, counters to zero, device error word cleared. Enqueued on `stream`. */
+gca_status gca_reset(gca_cache* cache, void* stream);
+
+/* Frees the host handle. Never frees the caller's workspace. NULL is accepted. */
+gca_status gca_cache_destroy(gca_cache* cache);
+
+/* Synchronises the device, reads the sticky device error word into the state and returns
+ * GCA_ERR_DEVICE if it is non-zero. */
+gca_status gca_check(gca_cache* cache);
+
+/* Fills *state from the host mirror (no GPU access). */
+gca_status gca_get_state(const gca_cache* cache, gca_state* state);
+
+/* Fills *info for the last gca_attend() call (host only). */
+gca_status gca_last_attend_info(const gca_cache* cache, gca_attend_info* info);
+
+/* Human-readable name of a status. */
+const char* gca_status_string(gca_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GCA_H_ */

@@ -1,0 +1,280 @@
+"""Python binding of libgca.so, the B200 paged KV cache for Geometric Context Attention.
+
+The functions below carry the C ABI's names (include/gca.h) and only marshal arguments;
+every step of the path runs in the library's CUDA kernels. PyTorch supplies device memory and
+streams. There is no fallback: if the library is missing or fails to load, the first call
+raises.
+
+`GcaCache` is a convenience owner of one cache: it allocates the workspace with torch, keeps
+the handle and exposes read-only tensor views of the device state for inspection.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "GcaError", "GcaConfig", "GcaState", "GcaAttendInfo", "lib", "library_path",
+    "gca_validate_config", "gca_workspace_bytes", "gca_cache_create", "gca_append_frame",
+    "gca_attend", "gca_reset", "gca_cache_destroy", "gca_check", "gca_get_state",
+    "gca_last_attend_info", "gca_status_string", "GcaCache", "config_for",
+    "EXPORTED_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def library_path() -> str:
+    return os.environ.get("GCA_LIBRARY", os.path.join(_HERE, "libgca.so"))
+
+
+GCA_OK = 0
+STATUS = {0: "GCA_OK", -1: "GCA_ERR_INVALID_ARG", -2: "GCA_ERR_OUT_OF_PAGES",
+          -3: "GCA_ERR_FRAME_ORDER", -4: "GCA_ERR_CUDA", -5: "GCA_ERR_UNSUPPORTED",
+          -6: "GCA_ERR_DEVICE"}
+
+
+class GcaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class GcaConfig(ctypes.Structure):
+    _fields_ = [
+        ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("page_size", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
+        ("num_special", ctypes.c_int32), ("anchor_frames", ctypes.c_int32),
+        ("window_frames", ctypes.c_int32), ("keep_tokens", ctypes.c_int32),
+        ("max_frames", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+        ("rope_base", ctypes.c_float),
+    ]
+
+
+class GcaState(ctypes.Structure):
+    _fields_ = [
+        ("frames_appended", ctypes.c_int64), ("free_head", ctypes.c_int64),
+        ("free_tail", ctypes.c_int64), ("traj_len", ctypes.c_int64),
+        ("traj_pages", ctypes.c_int32), ("tokens_per_frame", ctypes.c_int32),
+        ("pages_per_frame", ctypes.c_int32), ("pages_in_use", ctypes.c_int32),
+        ("device_error", ctypes.c_uint32), ("reserved", ctypes.c_int32),
+        ("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p),
+        ("free_ring", ctypes.c_void_p), ("frame_pages", ctypes.c_void_p),
+        ("traj_page_list", ctypes.c_void_p), ("slot_map", ctypes.c_void_p),
+        ("kept_tokens", ctypes.c_void_p),
+    ]
+
+
+class GcaAttendInfo(ctypes.Structure):
+    _fields_ = [
+        ("frame_idx", ctypes.c_int64), ("visible_keys", ctypes.c_int64),
+        ("logical_pages", ctypes.c_int32), ("kv_tiles", ctypes.c_int32),
+        ("query_tiles", ctypes.c_int32), ("grid", ctypes.c_int32), ("split", ctypes.c_int32),
+        ("launches", ctypes.c_int32),
+    ]
+
+
+# Every symbol include/gca.h declares.
+EXPORTED_SYMBOLS = (
+    "gca_validate_config", "gca_workspace_bytes", "gca_cache_create", "gca_append_frame",
+    "gca_attend", "gca_reset", "gca_cache_destroy", "gca_check", "gca_get_state",
+    "gca_last_attend_info", "gca_status_string",
+)
+
+_lib = None
+
+
+def lib():
+    """Loads libgca.so once. Raises if it is missing: there is no fallback path."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise ImportError(f"libgca.so not built ({path}); run "
+                          "`python -m paged_kv_cache_gca_b200.build`")
+    L = ctypes.CDLL(path)
+    P, I32, I64, SZ, VP = (ctypes.POINTER, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t,
+                           ctypes.c_void_p)
+    sig = {
+        "gca_validate_config": (I32, [P(GcaConfig)]),
+        "gca_workspace_bytes": (SZ, [P(GcaConfig)]),
+        "gca_cache_create": (I32, [P(GcaConfig), VP, SZ, VP, VP, P(VP)]),
+        "gca_append_frame": (I32, [VP, I64, VP, VP, VP, VP, VP]),
+        "gca_attend": (I32, [VP, I64, VP, VP, VP]),
+        "gca_reset": (I32, [VP, VP]),
+        "gca_cache_destroy": (I32, [VP]),
+        "gca_check": (I32, [VP]),
+        "gca_get_state": (I32, [VP, P(GcaState)]),
+        "gca_last_attend_info": (I32, [VP, P(GcaAttendInfo)]),
+        "gca_status_string": (ctypes.c_char_p, [I32]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _ok(status: int, where: str) -> None:
+    if status != GCA_OK:
+        raise GcaError(status, where)
+
+
+def gca_status_string(status: int) -> str:
+    return lib().gca_status_string(status).decode()
+
+
+def gca_validate_config(cfg: GcaConfig) -> int:
+    return lib().gca_validate_config(ctypes.byref(cfg))
+
+
+def gca_workspace_bytes(cfg: GcaConfig) -> int:
+    return lib().gca_workspace_bytes(ctypes.byref(cfg))
+
+
+def gca_cache_create(cfg: GcaConfig, workspace_ptr: int, workspace_bytes: int,
+                     initial_free_ptr: int | None, stream: int | None) -> int:
+    h = ctypes.c_void_p()
+    _ok(lib().gca_cache_create(ctypes.byref(cfg), workspace_ptr, workspace_bytes,
+                               initial_free_ptr, stream, ctypes.byref(h)), "gca_cache_create")
+    return h.value
+
+
+def gca_append_frame(handle, frame_idx, q_ptr, k_ptr, v_ptr, q_rot_ptr, stream) -> None:
+    _ok(lib().gca_append_frame(handle, frame_idx, q_ptr, k_ptr, v_ptr, q_rot_ptr, stream),
+        "gca_append_frame")
+
+
+def gca_attend(handle, frame_idx, q_rot_ptr, out_ptr, stream) -> None:
+    _ok(lib().gca_attend(handle, frame_idx, q_rot_ptr, out_ptr, stream), "gca_attend")
+
+
+def gca_reset(handle, stream) -> None:
+    _ok(lib().gca_reset(handle, stream), "gca_reset")
+
+
+def gca_cache_destroy(handle) -> None:
+    _ok(lib().gca_cache_destroy(handle), "gca_cache_destroy")
+
+
+def gca_check(handle) -> int:
+    return lib().gca_check(handle)
+
+
+def gca_get_state(handle) -> GcaState:
+    st = GcaState()
+    _ok(lib().gca_get_state(handle, ctypes.byref(st)), "gca_get_state")
+    return st
+
+
+def gca_last_attend_info(handle) -> GcaAttendInfo:
+    inf = GcaAttendInfo()
+    _ok(lib().gca_last_attend_info(handle, ctypes.byref(inf)), "gca_last_attend_info")
+    return inf
+
+
+def config_for(w, rope_base: float | None = None) -> GcaConfig:
+    """C config of a workload description (gca_inputs.Workload or anything with its fields)."""
+    return GcaConfig(num_heads=w.num_heads, head_dim=w.head_dim, page_size=w.page_size,
+                     grid_h=w.grid_h, grid_w=w.grid_w, num_special=w.num_special,
+                     anchor_frames=w.anchor_frames, window_frames=w.window_frames,
+                     keep_tokens=w.keep_tokens, max_frames=w.max_frames,
+                     num_pages=w.num_pages,
+                     rope_base=w.rope_base if rope_base is None else rope_base)
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+class GcaCache:
+    """One GCA cache on the current CUDA device, its workspace allocated by torch."""
+
+    def __init__(self, cfg: GcaConfig, initial_free=None, stream=None, device=None):
+        import torch
+
+        self.cfg = cfg
+        st = gca_validate_config(cfg)
+        _ok(st, "gca_validate_config")
+        self.nbytes = gca_workspace_bytes(cfg)
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        self.workspace = torch.empty(self.nbytes + 1024, dtype=torch.uint8, device=dev)
+        base = self.workspace.data_ptr()
+        self._off = (-base) % 1024
+        self._free = None
+        if initial_free is not None:
+            self._free = torch.as_tensor(initial_free, dtype=torch.int32).to(dev).contiguous()
+        self.handle = gca_cache_create(
+            cfg, base + self._off, self.nbytes,
+            None if self._free is None else self._free.data_ptr(), _stream_handle(stream))
+
+    def close(self):
+        if getattr(self, "handle", None):
+            gca_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ------------------------------------------------------------------ hot path
+    def append_frame(self, t, q, k, v, q_rot, stream=None):
+        gca_append_frame(self.handle, t, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                         q_rot.data_ptr(), _stream_handle(stream))
+
+    def attend(self, t, q_rot, out, stream=None):
+        gca_attend(self.handle, t, q_rot.data_ptr(), out.data_ptr(), _stream_handle(stream))
+
+    def reset(self, stream=None):
+        gca_reset(self.handle, _stream_handle(stream))
+
+    # ------------------------------------------------------------------ inspection
+    def check(self) -> int:
+        return gca_check(self.handle)
+
+    def state(self) -> GcaState:
+        return gca_get_state(self.handle)
+
+    def attend_info(self) -> GcaAttendInfo:
+        return gca_last_attend_info(self.handle)
+
+    def _view(self, ptr, count, dtype):
+        import torch
+
+        start = ptr - self.workspace.data_ptr()
+        nbytes = count * torch.empty((), dtype=dtype).element_size()
+        return self.workspace[start:start + nbytes].view(dtype)
+
+    def views(self):
+        """Device tensors over the cache state (no copies)."""
+        import torch
+
+        c, s = self.cfg, self.state()
+        ppf = s.pages_per_frame
+        page_shape = (c.num_pages, c.num_heads, c.page_size, c.head_dim)
+        n_page = c.num_pages * c.num_heads * c.page_size * c.head_dim
+        return {
+            "k_pool": self._view(s.k_pool, n_page, torch.bfloat16).view(page_shape),
+            "v_pool": self._view(s.v_pool, n_page, torch.bfloat16).view(page_shape),
+            "free_ring": self._view(s.free_ring, c.num_pages, torch.int32),
+            "frame_pages": self._view(s.frame_pages, c.max_frames * ppf,
+                                      torch.int32).view(c.max_frames, ppf),
+            "traj_pages": self._view(s.traj_page_list, max(s.traj_pages, 0), torch.int32),
+            "slot_map": self._view(s.slot_map, s.tokens_per_frame, torch.int32),
+            "kept_tokens": self._view(s.kept_tokens, c.keep_tokens, torch.int32),
+        }
+
+    def free_list(self):
+        """Free page ids in FIFO order (host list; synchronises)."""
+        s = self.state()
+        ring = self.views()["free_ring"].cpu().tolist()
+        n = self.cfg.num_pages
+        return [ring[i % n] for i in range(s.free_head, s.free_tail)]

@@ -1,0 +1,268 @@
+// Append-side kernels of the GCA paged KV cache (sm_100a).
+//
+// gca_append_kernel does one frame's whole append step in a single launch, following the order
+// of the pages' streaming block ("How the Geometric Context Transformer Enables Streaming 3D
+// Reconstruction in LingBot-Map", FlashInferBlock: append_frame, then evict_frames):
+//   a1  the frame's pages are popped from the FIFO free list (ring positions free_head ..
+//       free_head+ppf-1) and written to its page-table row; slot_map[i] = page*16 + i%16;
+//   a2  q and k get 3D (t, y, x) RoPE ("3D Rotary Positional Embeddings"); k_rot and v go to
+//       their slots with 16-byte stores, q_rot to the caller's buffer; the unused slots of the
+//       frame's last page are zeroed;
+//   a3  the frame leaving the window hands its kept tokens to the trajectory tail ("How GCT's
+//       Anchor-Pose-Trajectory Pools Make Monocular 3D Tractable": evicted frames keep only
+//       compact context tokens), new trajectory pages come from ring positions right after the
+//       frame's, and the evicted frame's pages go to the ring tail.
+// The host mirrors every count, so the ring positions are kernel arguments and no block waits
+// on another: the pops read positions [head, head+ppf+n_traj) while the pushes write
+// [tail, tail+ppf), and these never overlap because a frame is only evicted when at least
+// (A+W)*ppf pages are in use.
+#include <cuda_bf16.h>
+
+#include "gca_internal.h"
+
+namespace gca {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ void set_err(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
+
+__device__ __forceinline__ int ring_at(const int32_t* ring, int64_t pos, int32_t n) {
+  return ring[pos % n];
+}
+
+// ------------------------------------------------------------------------------- init
+
+__global__ void init_kernel(const InitParams p) {
+  const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  // free list and its saved copy; count occurrences for the permutation check
+  for (int64_t i = tid; i < p.num_pages; i += stride) {
+    int32_t v = p.user_free ? p.user_free[i] : (int32_t)i;
+    p.free_ring[i] = v;
+    p.init_free[i] = v;
+    if (v >= 0 && v < p.num_pages) {
+      atomicAdd(&p.seen[v], 1);
+    } else {
+      set_err(p.err, GCA_DEVERR_FREE_LIST);
+    }
+  }
+  for (int64_t i = tid; i < p.keep; i += stride) p.kept[i] = p.kept_host[i];
+  // RoPE tables in fp64, stored as fp32 (cos, sin): angle = pos * base^(-2j/d)
+  const int64_t n_t = (int64_t)p.max_frames * p.nt;
+  const int64_t n_y = (int64_t)(p.grid_h + 1) * p.ny;
+  const int64_t n_x = (int64_t)(p.grid_w + 1) * p.nx;
+  for (int64_t i = tid; i < n_t + n_y + n_x; i += stride) {
+    int64_t pos, j;
+    int d;
+    float2* dst;
+    if (i < n_t) {
+      pos = i / p.nt; j = i % p.nt; d = 2 * p.nt; dst = p.rope_t + i;
+    } else if (i < n_t + n_y) {
+      int64_t r = i - n_t;
+      pos = r / p.ny; j = r % p.ny; d = 2 * p.ny; dst = p.rope_y + r;
+    } else {
+      int64_t r = i - n_t - n_y;
+      pos = r / p.nx; j = r % p.nx; d = 2 * p.nx; dst = p.rope_x + r;
+    }
+    double inv_freq = pow(p.base, -2.0 * (double)j / (double)d);
+    double ang = (double)pos * inv_freq;
+    double sn, cs;
+    sincos(ang, &sn, &cs);
+    *dst = make_float2((float)cs, (float)sn);
+  }
+}
+
+__global__ void check_perm_kernel(const int32_t* seen, uint32_t* err, int32_t n) {
+  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i < n && seen[i] != 1) set_err(err, GCA_DEVERR_FREE_LIST);
+}
+
+__global__ void reset_kernel(int32_t* free_ring, const int32_t* init_free, uint32_t* err,
+                             int32_t n) {
+  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i < n) free_ring[i] = init_free[i];
+  if (i == 0) *err = 0u;
+}
+
+// ------------------------------------------------------------------------------- append
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+
+// Rotates the pair held in one 32-bit word (element 2j in the low half, 2j+1 in the high half).
+__device__ __forceinline__ uint32_t rotate_word(uint32_t w, float2 cs) {
+  const float a = bf_lo(w), b = bf_hi(w);
+  const float ra = fmaf(a, cs.x, -b * cs.y);
+  const float rb = fmaf(a, cs.y, b * cs.x);
+  return pack_bf2(ra, rb);
+}
+
+__global__ void __launch_bounds__(kThreads) append_kernel(const AppendParams p) {
+  const int64_t idx = blockIdx.x * (int64_t)kThreads + threadIdx.x;
+  if (idx >= p.n_items) return;
+  const int H = p.H;
+  const int64_t e_tok = p.n_tok_items;
+  const int64_t e_ev = e_tok + p.n_evict_items;
+  const int64_t e_zero = e_ev + p.n_zero_items;
+  const int64_t e_push = e_zero + p.n_push_items;
+
+  if (idx < e_tok) {
+    // ---- a1 + a2: one 16-byte chunk (8 dims) of one (token, head)
+    const int c = (int)(idx & 7);
+    const int64_t th = idx >> 3;
+    const int h = (int)(th % H);
+    const int i = (int)(th / H);
+    const int page = ring_at(p.free_ring, p.free_head + i / kPageSize, p.num_pages);
+    if (page < 0 || page >= p.num_pages) {
+      set_err(p.err, GCA_DEVERR_PAGE_RANGE);
+      return;
+    }
+    const int slot = i % kPageSize;
+    const int64_t dst = (((int64_t)page * H + h) * kPageSize + slot) * 8 + c;
+    if (h == 0 && c == 0) {
+      if (i < p.T) p.slot_map[i] = page * kPageSize + slot;
+      if (slot == 0) p.frame_pages[p.t * p.ppf + i / kPageSize] = page;
+    }
+    if (i >= p.T) {  // padding slot of the frame's last page
+      p.k_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
+      p.v_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
+      return;
+    }
+    const int64_t src = ((int64_t)i * H + h) * 8 + c;
+    const uint4 qv = p.q[src];
+    const uint4 kv = p.k[src];
+    const uint4 vv = p.v[src];
+    // positions: camera/register tokens at (t, 0, 0); patch (r, c) at (t, r+1, c+1)
+    int ypos = 0, xpos = 0;
+    if (i >= p.S) {
+      const int pidx = i - p.S;
+      ypos = pidx / p.grid_w + 1;
+      xpos = pidx % p.grid_w + 1;
+    }
+    float2 cs[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int j = 4 * c + w;  // pair index within the head
+      if (j < p.nt) {
+        cs[w] = p.rope_t[p.t * p.nt + j];
+      } else if (j < p.nt + p.ny) {
+        cs[w] = p.rope_y[ypos * p.ny + (j - p.nt)];
+      } else {
+        cs[w] = p.rope_x[xpos * p.nx + (j - p.nt - p.ny)];
+      }
+    }
+    uint4 qr, kr;
+    qr.x = rotate_word(qv.x, cs[0]);
+    qr.y = rotate_word(qv.y, cs[1]);
+    qr.z = rotate_word(qv.z, cs[2]);
+    qr.w = rotate_word(qv.w, cs[3]);
+    kr.x = rotate_word(kv.x, cs[0]);
+    kr.y = rotate_word(kv.y, cs[1]);
+    kr.z = rotate_word(kv.z, cs[2]);
+    kr.w = rotate_word(kv.w, cs[3]);
+    p.q_rot[src] = qr;
+    p.k_pool[dst] = kr;
+    p.v_pool[dst] = vv;
+    return;
+  }
+
+  if (idx < e_ev) {
+    // ---- a3: copy kept token j of the evicted frame to trajectory position traj_len + j
+    const int64_t r = idx - e_tok;
+    const int c = (int)(r & 7);
+    const int64_t th = r >> 3;
+    const int h = (int)(th % H);
+    const int j = (int)(th / H);
+    const int tok = p.kept[j];
+    const int src_page = p.frame_pages[(int64_t)p.evict_frame * p.ppf + tok / kPageSize];
+    const int64_t pos = p.traj_len + j;
+    const int64_t tp = pos / kPageSize;
+    const int dst_page =
+        tp < p.traj_pages_before
+            ? p.traj_pages[tp]
+            : ring_at(p.free_ring, p.free_head + p.ppf + (tp - p.traj_pages_before), p.num_pages);
+    if (src_page < 0 || src_page >= p.num_pages || dst_page < 0 || dst_page >= p.num_pages) {
+      set_err(p.err, GCA_DEVERR_PAGE_RANGE);
+      return;
+    }
+    const int64_t src = (((int64_t)src_page * H + h) * kPageSize + tok % kPageSize) * 8 + c;
+    const int64_t dst = (((int64_t)dst_page * H + h) * kPageSize + pos % kPageSize) * 8 + c;
+    p.k_pool[dst] = p.k_pool[src];
+    p.v_pool[dst] = p.v_pool[src];
+    return;
+  }
+
+  if (idx < e_zero) {
+    // ---- zero the slots of the last new trajectory page that this step leaves empty
+    const int64_t r = idx - e_ev;
+    const int c = (int)(r & 7);
+    const int64_t th = r >> 3;
+    const int h = (int)(th % H);
+    const int z = (int)(th / H);
+    const int64_t pos = p.traj_len + p.K + z;
+    const int64_t tp = pos / kPageSize;
+    const int page =
+        ring_at(p.free_ring, p.free_head + p.ppf + (tp - p.traj_pages_before), p.num_pages);
+    if (page < 0 || page >= p.num_pages) {
+      set_err(p.err, GCA_DEVERR_PAGE_RANGE);
+      return;
+    }
+    const int64_t dst = (((int64_t)page * H + h) * kPageSize + pos % kPageSize) * 8 + c;
+    p.k_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
+    p.v_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+
+  if (idx < e_push) {
+    // ---- push the evicted frame's pages to the free-list tail, in row order
+    const int k = (int)(idx - e_zero);
+    p.free_ring[(p.free_tail + k) % p.num_pages] =
+        p.frame_pages[(int64_t)p.evict_frame * p.ppf + k];
+    return;
+  }
+
+  // ---- record the trajectory pages popped by this step
+  const int k = (int)(idx - e_push);
+  p.traj_pages[p.traj_pages_before + k] =
+      ring_at(p.free_ring, p.free_head + p.ppf + k, p.num_pages);
+}
+
+}  // namespace
+
+cudaError_t launch_init(const InitParams& p, cudaStream_t s) {
+  int64_t work = p.num_pages;
+  int64_t rope = (int64_t)p.max_frames * p.nt + (int64_t)(p.grid_h + 1) * p.ny +
+                 (int64_t)(p.grid_w + 1) * p.nx;
+  if (rope > work) work = rope;
+  int64_t blocks = (work + kThreads - 1) / kThreads;
+  if (blocks > 4096) blocks = 4096;
+  if (blocks < 1) blocks = 1;
+  init_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_check_perm(int32_t* seen, uint32_t* err, int32_t n, cudaStream_t s) {
+  check_perm_kernel<<<(n + kThreads - 1) / kThreads, kThreads, 0, s>>>(seen, err, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reset(int32_t* free_ring, const int32_t* init_free, uint32_t* err,
+                         int32_t n, cudaStream_t s) {
+  reset_kernel<<<(n + kThreads - 1) / kThreads, kThreads, 0, s>>>(free_ring, init_free, err, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
+  const int64_t blocks = (p.n_items + kThreads - 1) / kThreads;
+  append_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace gca

@@ -1,0 +1,703 @@
+// Paged flash-attention forward for GCA on sm_100a (tcgen05 + TMEM + TMA).
+//
+// What it computes: for every head h and query row i of the last appended frame,
+//   out[i][h] = sum_j softmax_j(q_rot[i][h] . k_j[h] / sqrt(D)) v_j[h]
+// over the keys of the three pools -- anchor frame(s), the window of recent frames and the
+// trajectory pool ("LingBot-Map runs 10,000 frames on monocular video", section "How GCT's
+// Anchor-Pose-Trajectory Pools Make Monocular 3D Tractable"; "How the Geometric Context
+// Transformer Enables Streaming 3D Reconstruction in LingBot-Map", FlashInferBlock:
+// compute_attention). All of a frame's queries see the same key set (frame-causal attention,
+// same page, FAQ on scale frames), so the only mask is the one that hides unused page slots.
+//
+// Logical key order: anchor pages, window pages, trajectory pages; page lp -> physical page via
+// the page table. A 128-key tile is 8 pages; each page of one head is a contiguous 2 KB block
+// [16 slots][64 dims] bf16 that TMA copies into shared memory with the 128-byte swizzle.
+//
+// Work split: a (head, 128-query tile) pair is a unit; the flattened (unit, key tile) steps are
+// cut into `grid` equal ranges, one per CTA. A unit that spans several CTAs leaves partial
+// (O, row max, row sum) records that a combine kernel merges with log-sum-exp weights.
+//
+// CTA roles (192 threads):
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r). Loads Q into swizzled shared
+//              memory; per key tile reads S from TMEM, masks, does the online softmax in fp32
+//              with exp2, writes P (bf16) to TMEM, and rescales the O accumulator in TMEM only
+//              when the row max grows by more than 2^8 (lazy rescale). Epilogue writes O / l.
+//   warp 4     TMA producer: resolves the tile's 8 page ids and issues 16 page copies (K, V)
+//              per tile into a 3-stage ring.
+//   warp 5     MMA issuer (one thread): S = Q K^T (A, B from shared memory) into TMEM, then
+//              O += P V with P read from TMEM (A operand in tensor memory) and V from shared
+//              memory (MN-major). S of tile j+1 is issued before P V of tile j so the tensor
+//              core works while the softmax threads do.
+// TMEM (256 columns): S fp32 [0,128), P bf16x2 [128,192), O fp32 [192,256).
+// Every wait is bounded in time; on expiry the kernel sets GCA_DEVERR_WAIT_TIMEOUT, drains its
+// own copies, frees TMEM and returns.
+#include <cuda_bf16.h>
+
+#include "gca_internal.h"
+
+namespace gca {
+
+namespace {
+
+constexpr int kStages = 3;
+constexpr int kThreads = 192;
+constexpr int kWarpTma = 4;
+constexpr int kWarpMma = 5;
+constexpr uint32_t kTileBytes = kTileK * kHeadDim * 2;      // 16 KB
+constexpr uint32_t kPageBytes = kPageSize * kHeadDim * 2;    // 2 KB
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
+// Dynamic shared memory: Q tile, K and V stage rings (each 1024-byte aligned for the 128-byte
+// swizzle), then the barrier block. No static shared memory, so the dynamic base is the start
+// of the CTA's window (1024-aligned; checked at run time). Two CTAs fit in an SM's 228 KB.
+constexpr size_t kTilesBytes = (size_t)kTileBytes * (1 + 2 * kStages);
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
+constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale O when the max grows > 2^8
+
+struct __align__(8) Shared {
+  uint64_t k_full[kStages];
+  uint64_t v_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t q_full;
+  uint64_t s_full;
+  uint64_t s_free;
+  uint64_t p_full;
+  uint64_t pv_done;
+  uint64_t lens[kStages];  // 8 valid-slot counts (bytes) per stage
+  uint32_t tmem_base;
+  volatile int abort_flag;
+};
+constexpr size_t kSmemBytes = kTilesBytes + sizeof(Shared);
+
+// ------------------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+          smem_addr(bar)),
+      "r"(bytes)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete. Gives up when the CTA's abort flag is
+// set (unless `drain`) or after kWaitNs; a timeout sets the error bit and the abort flag.
+__device__ __noinline__ bool wait_phase(uint64_t* bar, uint32_t parity, Shared* sh,
+                                        uint32_t* err, bool drain = false) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0u) {
+      if (!drain && sh->abort_flag) return false;
+      if (global_timer() - t0 > kWaitNs) {
+        sh->abort_flag = 1;
+        atomicOr(err, GCA_DEVERR_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Every lane of the warp waits; the result is agreed across the warp so that warp-collective
+// instructions after it never run with diverged lanes.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Shared* sh,
+                                          uint32_t* err, bool drain = false) {
+  return __all_sync(0xffffffffu, wait_phase(bar, parity, sh, err, drain));
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Loads of 32 lanes x N consecutive 32-bit TMEM columns into registers, each followed by
+// tcgen05.wait::ld inside the same asm statement, so the compiler cannot schedule a use of the
+// registers before the data has arrived.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%128];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%129];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%130];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%131];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr + 0u), "r"(taddr + 32u), "r"(taddr + 64u), "r"(taddr + 96u)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr + 0u), "r"(taddr + 32u)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr + 0u)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 descriptor version 1).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // version
+  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, M = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major) {
+  return (1u << 4)                      // D fp32
+         | (1u << 7)                    // A bf16
+         | (1u << 10)                   // B bf16
+         | ((b_mn_major ? 1u : 0u) << 16)
+         | ((uint32_t)(n >> 3) << 17)
+         | ((uint32_t)(kTileQ >> 4) << 24);
+}
+
+// ------------------------------------------------------------------------- page walk
+
+// Physical page and valid-slot count of logical page lp (anchor, window, trajectory order).
+__device__ __forceinline__ void resolve_page(const AttnParams& p, int lp, int fallback,
+                                             int* page, int* len) {
+  if (lp < p.na_pages) {
+    *page = p.frame_pages[lp];
+    *len = (lp % p.ppf == p.ppf - 1) ? p.last_len : kPageSize;
+  } else if (lp < p.na_pages + p.nw_pages) {
+    const int w = lp - p.na_pages;
+    *page = p.frame_pages[p.win_base + w];
+    *len = (w % p.ppf == p.ppf - 1) ? p.last_len : kPageSize;
+  } else if (lp < p.n_lp) {
+    const int tp = lp - p.na_pages - p.nw_pages;
+    *page = p.traj_pages[tp];
+    *len = (tp == p.n_traj_pages - 1) ? p.traj_tail_len : kPageSize;
+  } else {
+    *page = fallback;  // any visible page: finite data, fully masked
+    *len = 0;
+  }
+}
+
+struct Segment {
+  int unit, j0, j1;
+};
+
+// ------------------------------------------------------------------------- kernel
+
+__global__ void __launch_bounds__(kThreads, 2)
+    attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                const AttnParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_addr(smem) & 1023u) != 0u) {  // the swizzled tiles need a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicOr(p.err, GCA_DEVERR_SMEM_ALIGN);
+    return;
+  }
+  Shared& sh = *reinterpret_cast<Shared*>(smem + kTilesBytes);
+  uint8_t* q_smem = smem;
+  uint8_t* k_smem = smem + kTileBytes;
+  uint8_t* v_smem = k_smem + kStages * kTileBytes;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh.k_full[s], 1);
+      mbar_init(&sh.v_full[s], 1);
+      mbar_init(&sh.kv_empty[s], 1);
+    }
+    mbar_init(&sh.q_full, kTileQ);
+    mbar_init(&sh.s_full, 1);
+    mbar_init(&sh.s_free, kTileQ);
+    mbar_init(&sh.p_full, kTileQ);
+    mbar_init(&sh.pv_done, 1);
+    sh.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpMma) {
+    asm volatile(
+        "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+            smem_addr(&sh.tmem_base)),
+        "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+
+  const int64_t s_begin = (int64_t)blockIdx.x * p.total / p.grid;
+  const int64_t s_end = (int64_t)(blockIdx.x + 1) * p.total / p.grid;
+
+  if (warp == kWarpTma) {
+    // ------------------------------------------------------------ TMA producer
+    int fallback = 0;
+    int flen = 0;
+    resolve_page(p, 0, 0, &fallback, &flen);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int64_t s = s_begin; s < s_end && ok;) {
+      const int u = (int)(s / p.n_tiles);
+      const int64_t seg_end = min(s_end, (int64_t)(u + 1) * p.n_tiles);
+      const int h = u / p.n_qt;
+      for (int j = (int)(s - (int64_t)u * p.n_tiles); j < (int)(seg_end - (int64_t)u * p.n_tiles);
+           ++j, ++it) {
+        const int stage = it % kStages;
+        const uint32_t use = it / kStages;
+        if (use > 0 && !warp_wait(&sh.kv_empty[stage], (use - 1) & 1u, &sh, p.err)) {
+          ok = false;
+          break;
+        }
+        int page = 0, len = 0;
+        if (lane < kPagesPerTile) resolve_page(p, j * kPagesPerTile + lane, fallback, &page, &len);
+        if (page < 0 || page >= p.num_pages) {
+          atomicOr(p.err, GCA_DEVERR_PAGE_RANGE);
+          page = 0;
+          len = 0;
+        }
+        uint64_t lens = 0;
+#pragma unroll
+        for (int k = 0; k < kPagesPerTile; ++k) {
+          lens |= (uint64_t)(uint32_t)__shfl_sync(0xffffffffu, len, k) << (8 * k);
+        }
+        if (lane == 0) {
+          sh.lens[stage] = lens;
+          mbar_arrive_expect_tx(&sh.k_full[stage], kTileBytes);
+          mbar_arrive_expect_tx(&sh.v_full[stage], kTileBytes);
+        }
+        __syncwarp();
+        if (lane < kPagesPerTile) {
+          const int row = (page * p.H + h) * kPageSize;
+          tma_load_2d(smem_addr(k_smem + stage * kTileBytes + lane * kPageBytes), &tm_k, 0, row,
+                      &sh.k_full[stage]);
+          tma_load_2d(smem_addr(v_smem + stage * kTileBytes + lane * kPageBytes), &tm_v, 0, row,
+                      &sh.v_full[stage]);
+        }
+      }
+      s = seg_end;
+    }
+    // Drain: wait until the last issued copies have landed before the CTA can exit.
+    const uint32_t issued = it;
+    const uint32_t first = issued > (uint32_t)kStages ? issued - kStages : 0u;
+    for (uint32_t q = first; q < issued; ++q) {
+      const int stage = q % kStages;
+      const uint32_t use = q / kStages;
+      warp_wait(&sh.k_full[stage], use & 1u, &sh, p.err, true);
+      warp_wait(&sh.v_full[stage], use & 1u, &sh, p.err, true);
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = idesc_bf16(kTileK, false);
+      constexpr uint32_t kIdescPV = idesc_bf16(kHeadDim, true);
+      const uint64_t q_desc = sw128_desc(smem_addr(q_smem), 16, 1024);
+      uint32_t it = 0, seg = 0;
+      bool ok = true;
+      for (int64_t s = s_begin; s < s_end && ok; ++seg) {
+        const int u = (int)(s / p.n_tiles);
+        const int64_t seg_end = min(s_end, (int64_t)(u + 1) * p.n_tiles);
+        const int j0 = (int)(s - (int64_t)u * p.n_tiles);
+        const int j1 = (int)(seg_end - (int64_t)u * p.n_tiles);
+        if (!wait_phase(&sh.q_full, seg & 1u, &sh, p.err)) break;
+        tc_fence_after();
+        for (int j = j0; j < j1; ++j, ++it) {
+          const int stage = it % kStages;
+          const uint32_t use = it / kStages;
+          if (!wait_phase(&sh.k_full[stage], use & 1u, &sh, p.err)) { ok = false; break; }
+          if (j > j0 && !wait_phase(&sh.s_free, (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t k_desc = sw128_desc(smem_addr(k_smem + stage * kTileBytes), 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+            // +32 bytes along K inside the swizzled 128-byte rows
+            mma_ss(tmem + kColS, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&sh.s_full);
+          if (j > j0) {
+            const uint32_t pit = it - 1;
+            const int pst = pit % kStages;
+            if (!wait_phase(&sh.p_full, pit & 1u, &sh, p.err)) { ok = false; break; }
+            if (!wait_phase(&sh.v_full[pst], (pit / kStages) & 1u, &sh, p.err)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t v_desc = sw128_desc(smem_addr(v_smem + pst * kTileBytes), 16384, 1024);
+#pragma unroll
+            for (int kk = 0; kk < kTileK / 16; ++kk) {
+              // 16 keys = 2048 bytes of V; 8 TMEM columns of packed P
+              mma_ts(tmem + kColO, tmem + kColP + 8 * kk, v_desc + 128 * kk, kIdescPV,
+                     (j - 1 > j0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&sh.pv_done);
+            mma_commit(&sh.kv_empty[pst]);
+          }
+        }
+        if (!ok) break;
+        // P V of the segment's last tile
+        const uint32_t pit = it - 1;
+        const int pst = pit % kStages;
+        if (!wait_phase(&sh.p_full, pit & 1u, &sh, p.err)) break;
+        if (!wait_phase(&sh.v_full[pst], (pit / kStages) & 1u, &sh, p.err)) break;
+        tc_fence_after();
+        const uint64_t v_desc = sw128_desc(smem_addr(v_smem + pst * kTileBytes), 16384, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kTileK / 16; ++kk) {
+          mma_ts(tmem + kColO, tmem + kColP + 8 * kk, v_desc + 128 * kk, kIdescPV,
+                 (j1 - 1 > j0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&sh.pv_done);
+        mma_commit(&sh.kv_empty[pst]);
+        s = seg_end;
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warps 0-3
+    const int r = threadIdx.x;  // query row within the tile == TMEM lane
+    const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int64_t s = s_begin; s < s_end && ok;) {
+      const int u = (int)(s / p.n_tiles);
+      const int64_t seg_end = min(s_end, (int64_t)(u + 1) * p.n_tiles);
+      const int j0 = (int)(s - (int64_t)u * p.n_tiles);
+      const int j1 = (int)(seg_end - (int64_t)u * p.n_tiles);
+      const int h = u / p.n_qt;
+      const int qt = u % p.n_qt;
+      const int qi = qt * kTileQ + r;
+
+      // Q row -> shared memory, 128-byte swizzle (16-byte chunk c of row r at c ^ (r % 8))
+      {
+        const uint4* src = p.q + ((int64_t)qi * p.H + h) * 8;
+        uint8_t* row = q_smem + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 v = qi < p.T ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&sh.q_full);
+      }
+
+      float m_run = -INFINITY;  // running row max, log2 units (scaled)
+      float l_run = 0.f;        // running row sum relative to m_run
+      for (int j = j0; j < j1; ++j, ++it) {
+        if (!warp_wait(&sh.s_full, it & 1u, &sh, p.err)) { ok = false; break; }
+        tc_fence_after();
+        float sv[kTileK];
+        tmem_ld128(t_row + kColS, sv);
+        tc_fence_before();
+        mbar_arrive(&sh.s_free);
+
+        const int stage = it % kStages;
+        if (!warp_wait(&sh.k_full[stage], (it / kStages) & 1u, &sh, p.err)) { ok = false; break; }
+        const uint64_t lens = sh.lens[stage];
+        if (lens != 0x1010101010101010ull) {
+#pragma unroll
+          for (int pg = 0; pg < kPagesPerTile; ++pg) {
+            const int len = (int)((lens >> (8 * pg)) & 0xffu);
+            if (len < kPageSize) {
+#pragma unroll
+              for (int c = 0; c < kPageSize; ++c) {
+                if (c >= len) sv[pg * kPageSize + c] = -INFINITY;
+              }
+            }
+          }
+        }
+        // row max
+        float mx[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx[a] = sv[a];
+#pragma unroll
+        for (int c = 8; c < kTileK; c += 8) {
+#pragma unroll
+          for (int a = 0; a < 8; ++a) mx[a] = fmaxf(mx[a], sv[c + a]);
+        }
+        const float tile_max =
+            fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+            p.scale_log2;
+        float m_new = m_run, alpha = 1.f;
+        if (tile_max > m_run + kRescaleThreshold) {
+          m_new = tile_max;
+          alpha = ex2(m_run - m_new);
+        }
+        // p = 2^(s*c - m), row sum
+        float rs[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) rs[a] = 0.f;
+#pragma unroll
+        for (int c = 0; c < kTileK; c += 8) {
+#pragma unroll
+          for (int a = 0; a < 8; ++a) {
+            const float e = ex2(fmaf(sv[c + a], p.scale_log2, -m_new));
+            sv[c + a] = e;
+            rs[a] += e;
+          }
+        }
+        const float row_sum =
+            ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+
+        if (j > j0) {
+          // P V of the previous tile must be done before P is overwritten or O rescaled
+          if (!warp_wait(&sh.pv_done, (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+            for (int c = 0; c < kHeadDim / 16; ++c) {
+              float o[16];
+              tmem_ld16(t_row + kColO + 16 * c, o);
+#pragma unroll
+              for (int a = 0; a < 16; ++a) o[a] *= alpha;
+              tmem_st16(t_row + kColO + 16 * c, o);
+            }
+            tmem_wait_st();
+          }
+        }
+        l_run = l_run * alpha + row_sum;
+        m_run = m_new;
+
+        uint32_t pk[kTileK / 2];
+#pragma unroll
+        for (int c = 0; c < kTileK / 2; ++c) pk[c] = pack_bf2(sv[2 * c], sv[2 * c + 1]);
+        tmem_st32(t_row + kColP, pk);
+        tmem_st32(t_row + kColP + 32, pk + 32);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sh.p_full);
+      }
+      if (!ok) break;
+
+      // ---- epilogue
+      if (!warp_wait(&sh.pv_done, (it - 1) & 1u, &sh, p.err)) break;
+      tc_fence_after();
+      float o[kHeadDim];
+      tmem_ld64(t_row + kColO, o);
+      tc_fence_before();
+      if (j0 == 0 && j1 == p.n_tiles) {
+        if (qi < p.T) {
+          const float inv = 1.f / l_run;
+          uint4* dst = p.out + ((int64_t)qi * p.H + h) * 8;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 w;
+            w.x = pack_bf2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
+            w.y = pack_bf2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
+            w.z = pack_bf2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
+            w.w = pack_bf2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
+            dst[c] = w;
+          }
+        }
+      } else {
+        const int64_t slot = (int64_t)blockIdx.x + u;
+        float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * kTileQ + r) * kHeadDim);
+#pragma unroll
+        for (int c = 0; c < kHeadDim / 4; ++c) {
+          dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        }
+        p.part_ml[slot * kTileQ + r] = make_float2(m_run, l_run);
+      }
+      s = seg_end;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols));
+  }
+}
+
+// Merges the partial records of every split unit: weights 2^(m_s - M), M = max_s m_s.
+__global__ void __launch_bounds__(kTileQ) combine_kernel(const AttnParams p) {
+  const int u = blockIdx.x;
+  const int r = threadIdx.x;
+  const int64_t first = (int64_t)u * p.n_tiles;
+  const int64_t c0 = cta_of_step(first, p.total, p.grid);
+  const int64_t c1 = cta_of_step(first + p.n_tiles - 1, p.total, p.grid);
+  if (c0 == c1) return;
+  const int h = u / p.n_qt;
+  const int qi = (u % p.n_qt) * kTileQ + r;
+  if (qi >= p.T) return;
+  float M = -INFINITY;
+  for (int64_t c = c0; c <= c1; ++c) M = fmaxf(M, p.part_ml[(c + u) * kTileQ + r].x);
+  float acc[kHeadDim];
+#pragma unroll
+  for (int a = 0; a < kHeadDim; ++a) acc[a] = 0.f;
+  float L = 0.f;
+  for (int64_t c = c0; c <= c1; ++c) {
+    const float2 ml = p.part_ml[(c + u) * kTileQ + r];
+    const float w = ex2(ml.x - M);
+    L += w * ml.y;
+    const float4* src = reinterpret_cast<const float4*>(p.part_o + ((c + u) * kTileQ + r) * kHeadDim);
+#pragma unroll
+    for (int a = 0; a < kHeadDim / 4; ++a) {
+      const float4 v = src[a];
+      acc[4 * a] += w * v.x;
+      acc[4 * a + 1] += w * v.y;
+      acc[4 * a + 2] += w * v.z;
+      acc[4 * a + 3] += w * v.w;
+    }
+  }
+  const float inv = 1.f / L;
+  uint4* dst = p.out + ((int64_t)qi * p.H + h) * 8;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 w;
+    w.x = pack_bf2(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
+    w.y = pack_bf2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
+    w.z = pack_bf2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
+    w.w = pack_bf2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
+    dst[c] = w;
+  }
+}
+
+}  // namespace
+
+cudaError_t attn_prepare(int* ctas_per_sm) {
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  int n = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel, kThreads, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  // Two CTAs share the SM's 512 TMEM columns (256 each); never more.
+  *ctas_per_sm = n < 1 ? 1 : (n > 2 ? 2 : n);
+  return cudaSuccess;
+}
+
+cudaError_t launch_attn(const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
+                        cudaStream_t s) {
+  attn_kernel<<<p.grid, kThreads, kSmemBytes, s>>>(tk, tv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const AttnParams& p, cudaStream_t s) {
+  combine_kernel<<<p.units, kTileQ, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace gca

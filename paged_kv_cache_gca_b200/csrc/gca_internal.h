@@ -1,0 +1,141 @@
+// Internal declarations shared by the host API (gca_api.cu) and the kernels
+// (gca_append.cu, gca_attn.cu). Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/gca.h"
+
+namespace gca {
+
+constexpr int kHeadDim = 64;
+constexpr int kPageSize = 16;
+constexpr int kMaxHeads = 64;
+constexpr int kMaxKeep = 64;
+constexpr int kTileQ = 128;     // query rows per attention tile
+constexpr int kTileK = 128;     // keys per attention tile (8 pages)
+constexpr int kPagesPerTile = kTileK / kPageSize;
+constexpr int kMaxGrid = 512;   // attention CTAs per launch (sizes the split buffers)
+constexpr size_t kAlign = 1024;
+
+// Byte offsets of every region inside the caller's workspace.
+struct Layout {
+  size_t k_pool, v_pool;     // bf16 [num_pages][H][16][64]
+  size_t free_ring;          // int32 [num_pages]
+  size_t init_free;          // int32 [num_pages] (restored by reset)
+  size_t seen;               // int32 [num_pages] (permutation check at create)
+  size_t frame_pages;        // int32 [max_frames][ppf]
+  size_t traj_pages;         // int32 [traj_cap_pages]
+  size_t slot_map;           // int32 [T]
+  size_t kept;               // int32 [kMaxKeep]
+  size_t rope_t, rope_y, rope_x;  // float2 (cos, sin) tables
+  size_t err;                // uint32 sticky device error word
+  size_t part_o;             // float [part_slots][128][64]
+  size_t part_ml;            // float2 [part_slots][128]
+  size_t total;
+  int64_t traj_cap_pages;
+  int32_t part_slots;
+  int32_t T, ppf, last_len;  // tokens per frame, pages per frame, valid slots of the last page
+  int32_t n_qt;              // query tiles per head
+  int32_t nt, ny, nx;        // RoPE pairs per band (t, y, x)
+};
+
+bool compute_layout(const gca_config& cfg, Layout* lay);
+void kept_token_list(const gca_config& cfg, int32_t* out, int32_t* count);
+
+// ---------------------------------------------------------------------- kernels' arguments
+
+struct InitParams {
+  int32_t* free_ring;
+  int32_t* init_free;
+  int32_t* seen;
+  const int32_t* user_free;  // may be null
+  int32_t* kept;
+  float2* rope_t;
+  float2* rope_y;
+  float2* rope_x;
+  uint32_t* err;
+  int32_t num_pages;
+  int32_t max_frames, grid_h, grid_w;
+  int32_t nt, ny, nx;
+  int32_t keep;
+  double base;
+  int32_t kept_host[kMaxKeep];
+};
+
+struct AppendParams {
+  const uint4* q;
+  const uint4* k;
+  const uint4* v;
+  uint4* q_rot;
+  uint4* k_pool;
+  uint4* v_pool;
+  int32_t* free_ring;
+  int32_t* frame_pages;
+  int32_t* traj_pages;
+  int32_t* slot_map;
+  const int32_t* kept;
+  const float2* rope_t;
+  const float2* rope_y;
+  const float2* rope_x;
+  uint32_t* err;
+  int64_t t;
+  int64_t free_head;
+  int64_t free_tail;
+  int64_t traj_len;
+  int32_t T, H, S, grid_w, ppf, num_pages;
+  int32_t nt, ny, nx;
+  int32_t evict_frame;        // -1: nothing leaves the window
+  int32_t K;                  // kept tokens copied (0 if no eviction)
+  int32_t traj_pages_before;  // trajectory pages before this step
+  int32_t n_pop_traj;         // trajectory pages popped by this step
+  int32_t zero_slots;         // slots zero-filled at the end of the last new trajectory page
+  // item ranges of the single launch
+  int64_t n_tok_items, n_evict_items, n_zero_items, n_push_items, n_traj_items, n_items;
+};
+
+struct AttnParams {
+  const uint4* q;        // rotated queries [T][H][64] bf16
+  uint4* out;            // [T][H][64] bf16
+  float* part_o;         // [slots][128][64]
+  float2* part_ml;       // [slots][128] (row max in log2 units, row sum)
+  const int32_t* frame_pages;
+  const int32_t* traj_pages;
+  uint32_t* err;
+  int32_t T, H, ppf, last_len, num_pages;
+  int32_t na_pages;      // anchor pages (visible anchor frames * ppf)
+  int32_t win_base;      // index into frame_pages of the first window page
+  int32_t nw_pages;      // window pages
+  int32_t n_traj_pages;
+  int32_t traj_tail_len; // valid slots of the last trajectory page
+  int32_t n_lp;          // logical pages walked
+  int32_t n_tiles;       // 128-key tiles
+  int32_t n_qt;          // 128-query tiles per head
+  int32_t units;         // H * n_qt
+  int64_t total;         // units * n_tiles
+  int32_t grid;
+  float scale_log2;      // log2(e) / sqrt(D)
+};
+
+// Launchers (return cudaGetLastError() of the launch).
+cudaError_t launch_init(const InitParams& p, cudaStream_t s);
+cudaError_t launch_check_perm(int32_t* seen, uint32_t* err, int32_t n, cudaStream_t s);
+cudaError_t launch_reset(int32_t* free_ring, const int32_t* init_free, uint32_t* err,
+                         int32_t n, cudaStream_t s);
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+cudaError_t attn_prepare(int* ctas_per_sm);  // sets kernel attributes, reports occupancy
+cudaError_t launch_attn(const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
+                        cudaStream_t s);
+cudaError_t launch_combine(const AttnParams& p, cudaStream_t s);
+
+// Split bookkeeping shared by the attention and combine kernels: CTA c owns the flattened
+// (unit, tile) steps [c*total/grid, (c+1)*total/grid); the CTA that holds step s is
+// ceil((s+1)*grid/total) - 1, and (unit u, CTA c) writes its partial result to slot c + u.
+__host__ __device__ inline int64_t cta_of_step(int64_t s, int64_t total, int64_t grid) {
+  return ((s + 1) * grid + total - 1) / total - 1;
+}
+
+}  // namespace gca

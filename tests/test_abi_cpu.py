@@ -1,0 +1,103 @@
+"""The C-ABI library builds, loads and exports every symbol include/gca.h declares; host-only
+entry points (validation, workspace sizing, status names) work without a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import gca_inputs as gi
+import paged_kv_cache_gca_b200 as gca
+from paged_kv_cache_gca_b200 import build as gbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return gca.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "gca.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gca_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert header_functions() == sorted(gca.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_header_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", gca.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in header_functions():
+        assert name in exported, name
+        assert getattr(L, name) is not None
+
+
+def test_library_is_sm100a(L):
+    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", gca.library_path()],
+                         capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    assert "sm_100a" in out.stdout
+
+
+def test_status_strings(L):
+    for code, name in gca.STATUS.items():
+        assert gca.gca_status_string(code) == name
+
+
+@pytest.mark.parametrize("name", list(gi.WORKLOADS))
+def test_workloads_validate_and_size(L, name):
+    w = gi.workload(name)
+    cfg = gca.config_for(w)
+    assert gca.gca_validate_config(cfg) == 0
+    n = gca.gca_workspace_bytes(cfg)
+    pools = 2 * w.num_pages * w.num_heads * w.page_size * w.head_dim * 2
+    assert pools < n < pools + 64 * 2**20 + 8 * w.max_frames * 64
+    assert n % 1024 == 0
+
+
+def test_invalid_configs(L):
+    base = gca.config_for(gi.workload("w16_320"))
+
+    def with_(**kw):
+        c = gca.GcaConfig()
+        ctypes.memmove(ctypes.byref(c), ctypes.byref(base), ctypes.sizeof(c))
+        for k, v in kw.items():
+            setattr(c, k, v)
+        return c
+
+    assert gca.gca_validate_config(with_(window_frames=0)) == -1
+    assert gca.gca_validate_config(with_(num_heads=0)) == -1
+    assert gca.gca_validate_config(with_(keep_tokens=2000)) == -1
+    assert gca.gca_validate_config(with_(rope_base=-1.0)) == -1
+    assert gca.gca_validate_config(with_(num_pages=0)) == -1
+    assert gca.gca_validate_config(with_(head_dim=128)) == -5
+    assert gca.gca_validate_config(with_(page_size=32)) == -5
+    assert gca.gca_validate_config(with_(keep_tokens=80)) == -5
+    assert gca.gca_workspace_bytes(with_(window_frames=0)) == 0
+    assert L.gca_validate_config(None) == -1
+
+
+def test_create_rejects_bad_arguments_before_touching_cuda(L):
+    cfg = gca.config_for(gi.workload("tiny"))
+    h = ctypes.c_void_p()
+    n = gca.gca_workspace_bytes(cfg)
+    # null out-pointer, null workspace, misaligned workspace, too-small workspace
+    assert L.gca_cache_create(ctypes.byref(cfg), 1024, n, None, None, None) == -1
+    assert L.gca_cache_create(ctypes.byref(cfg), None, n, None, None, ctypes.byref(h)) == -1
+    assert L.gca_cache_create(ctypes.byref(cfg), 1024 + 16, n, None, None, ctypes.byref(h)) == -1
+    assert L.gca_cache_create(ctypes.byref(cfg), 1024, n - 1, None, None, ctypes.byref(h)) == -1
+    assert h.value is None
+    # calls on a null handle
+    assert L.gca_append_frame(None, 0, 1, 1, 1, 1, None) == -1
+    assert L.gca_attend(None, 0, 1, 1, None) == -1
+    assert L.gca_reset(None, None) == -1
+    assert L.gca_check(None) == -1
+    assert L.gca_cache_destroy(None) == 0
