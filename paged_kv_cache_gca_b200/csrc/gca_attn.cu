@@ -112,7 +112,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Waits for the phase with the given parity to complete. Gives up when the CTA's abort flag is
 // set (unless `drain`) or after kWaitNs; a timeout sets the error bit and the abort flag.
-__device__ __noinline__ bool wait_phase(uint64_t* bar, uint32_t parity, Shared* sh,
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, Shared* sh,
                                         uint32_t* err, bool drain = false) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer();
@@ -578,11 +578,15 @@ __global__ void __launch_bounds__(kThreads, 2)
         l_run = l_run * alpha + row_sum;
         m_run = m_new;
 
-        uint32_t pk[kTileK / 2];
 #pragma unroll
-        for (int c = 0; c < kTileK / 2; ++c) pk[c] = pack_bf2(sv[2 * c], sv[2 * c + 1]);
-        tmem_st32(t_row + kColP, pk);
-        tmem_st32(t_row + kColP + 32, pk + 32);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[kTileK / 4];
+#pragma unroll
+          for (int c = 0; c < kTileK / 4; ++c) {
+            pk[c] = pack_bf2(sv[64 * half + 2 * c], sv[64 * half + 2 * c + 1]);
+          }
+          tmem_st32(t_row + kColP + 32 * half, pk);
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sh.p_full);
@@ -680,6 +684,9 @@ __global__ void __launch_bounds__(kTileQ) combine_kernel(const AttnParams p) {
 cudaError_t attn_prepare(int* ctas_per_sm) {
   cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   int n = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel, kThreads, kSmemBytes);
