@@ -35,6 +35,25 @@
 
 #include "gca_internal.h"
 
+// Softmax arithmetic options (defaults are the measured best on B200):
+//   GCA_EXP_BF16  1: P = ex2.bf16x2(bf16(s*c - m)) (two exponentials per MUFU issue);
+//                 0: fp32 ex2 per element, then rounded to bf16 pairs.
+//   GCA_FMA2      1: scale-subtract with packed f32x2 FMA; 0: scalar FMA.
+//   GCA_SUM_MIXED 1: row sum with mixed-precision bf16 -> fp32 adds; 0: plain fp32 adds.
+//   GCA_MAX_CHAINS independent 3-input max chains (4 or 8).
+#ifndef GCA_EXP_BF16
+#define GCA_EXP_BF16 0
+#endif
+#ifndef GCA_FMA2
+#define GCA_FMA2 0
+#endif
+#ifndef GCA_SUM_MIXED
+#define GCA_SUM_MIXED 1
+#endif
+#ifndef GCA_MAX_CHAINS
+#define GCA_MAX_CHAINS 4
+#endif
+
 namespace gca {
 
 namespace {
@@ -46,6 +65,7 @@ constexpr int kWarpMma = 5;
 constexpr uint32_t kTileBytes = kTileK * kHeadDim * 2;      // 16 KB
 constexpr uint32_t kPageBytes = kPageSize * kHeadDim * 2;    // 2 KB
 constexpr uint32_t kTmemCols = 256;
+// TMEM columns: S fp32 [0,128), P bf16x2 [128,192), O fp32 [192,256).
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
 // Dynamic shared memory: Q tile, K and V stage rings (each 1024-byte aligned for the 128-byte
 // swizzle), then the barrier block. No static shared memory, so the dynamic base is the start
@@ -252,6 +272,46 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 instructions): one issue slot for two lanes of math.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on both bf16 halves (MUFU, two results per issue).
+__device__ __forceinline__ uint32_t ex2_bf2(uint32_t x) {
+  uint32_t y;
+  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// acc_lo += low bf16 half of w, acc_hi += high half (mixed-precision adds, fp32 result).
+__device__ __forceinline__ void add_bf2(float& acc_lo, float& acc_hi, uint32_t w) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(acc_lo), "+f"(acc_hi)
+      : "r"(w));
+}
+
 __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
   __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&b);
@@ -410,6 +470,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
+    // Per tile j: S(j) = Q K_j^T is issued as soon as the softmax warps have read S(j-1) out of
+    // TMEM, so it runs while they compute P(j-1); then O += P(j-1) V_(j-1).
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16(kTileK, false);
       constexpr uint32_t kIdescPV = idesc_bf16(kHeadDim, true);
@@ -423,21 +485,23 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int j1 = (int)(seg_end - (int64_t)u * p.n_tiles);
         if (!wait_phase(&sh.q_full, seg & 1u, &sh, p.err)) break;
         tc_fence_after();
-        for (int j = j0; j < j1; ++j, ++it) {
-          const int stage = it % kStages;
-          const uint32_t use = it / kStages;
-          if (!wait_phase(&sh.k_full[stage], use & 1u, &sh, p.err)) { ok = false; break; }
-          if (j > j0 && !wait_phase(&sh.s_free, (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t k_desc = sw128_desc(smem_addr(k_smem + stage * kTileBytes), 16, 1024);
+        for (int j = j0; j <= j1; ++j) {
+          if (j < j1) {
+            const int stage = it % kStages;
+            const uint32_t use = it / kStages;
+            if (!wait_phase(&sh.k_full[stage], use & 1u, &sh, p.err)) { ok = false; break; }
+            if (j > j0 && !wait_phase(&sh.s_free, (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t k_desc = sw128_desc(smem_addr(k_smem + stage * kTileBytes), 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-            // +32 bytes along K inside the swizzled 128-byte rows
-            mma_ss(tmem + kColS, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+              // +32 bytes along K inside the swizzled 128-byte rows
+              mma_ss(tmem + kColS, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&sh.s_full);
           }
-          mma_commit(&sh.s_full);
           if (j > j0) {
-            const uint32_t pit = it - 1;
+            const uint32_t pit = it - 1;  // tile j-1
             const int pst = pit % kStages;
             if (!wait_phase(&sh.p_full, pit & 1u, &sh, p.err)) { ok = false; break; }
             if (!wait_phase(&sh.v_full[pst], (pit / kStages) & 1u, &sh, p.err)) { ok = false; break; }
@@ -445,29 +509,15 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint64_t v_desc = sw128_desc(smem_addr(v_smem + pst * kTileBytes), 16384, 1024);
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk) {
-              // 16 keys = 2048 bytes of V; 8 TMEM columns of packed P
+              // 16 keys: 2048 bytes of V, 8 TMEM columns of packed P
               mma_ts(tmem + kColO, tmem + kColP + 8 * kk, v_desc + 128 * kk, kIdescPV,
                      (j - 1 > j0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(&sh.pv_done);
             mma_commit(&sh.kv_empty[pst]);
           }
+          if (j < j1) ++it;
         }
-        if (!ok) break;
-        // P V of the segment's last tile
-        const uint32_t pit = it - 1;
-        const int pst = pit % kStages;
-        if (!wait_phase(&sh.p_full, pit & 1u, &sh, p.err)) break;
-        if (!wait_phase(&sh.v_full[pst], (pit / kStages) & 1u, &sh, p.err)) break;
-        tc_fence_after();
-        const uint64_t v_desc = sw128_desc(smem_addr(v_smem + pst * kTileBytes), 16384, 1024);
-#pragma unroll
-        for (int kk = 0; kk < kTileK / 16; ++kk) {
-          mma_ts(tmem + kColO, tmem + kColP + 8 * kk, v_desc + 128 * kk, kIdescPV,
-                 (j1 - 1 > j0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&sh.pv_done);
-        mma_commit(&sh.kv_empty[pst]);
         s = seg_end;
       }
     }
@@ -508,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         float sv[kTileK];
         tmem_ld128(t_row + kColS, sv);
         tc_fence_before();
-        mbar_arrive(&sh.s_free);
+        mbar_arrive(&sh.s_free);  // the MMA warp may now compute the next S
 
         const int stage = it % kStages;
         if (!warp_wait(&sh.k_full[stage], (it / kStages) & 1u, &sh, p.err)) { ok = false; break; }
@@ -525,37 +575,63 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
           }
         }
-        // row max
-        float mx[8];
+        // row max: independent chains of 3-input max
+        constexpr int kCh = GCA_MAX_CHAINS;
+        float mx[kCh];
 #pragma unroll
-        for (int a = 0; a < 8; ++a) mx[a] = sv[a];
+        for (int a = 0; a < kCh; ++a) mx[a] = fmaxf(sv[2 * a], sv[2 * a + 1]);
 #pragma unroll
-        for (int c = 8; c < kTileK; c += 8) {
+        for (int c = 2 * kCh; c < kTileK; c += 2 * kCh) {
 #pragma unroll
-          for (int a = 0; a < 8; ++a) mx[a] = fmaxf(mx[a], sv[c + a]);
+          for (int a = 0; a < kCh; ++a) mx[a] = max3(mx[a], sv[c + 2 * a], sv[c + 2 * a + 1]);
         }
-        const float tile_max =
-            fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                  fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
-            p.scale_log2;
+#pragma unroll
+        for (int w = kCh / 2; w >= 1; w /= 2) {
+#pragma unroll
+          for (int a = 0; a < w; ++a) mx[a] = fmaxf(mx[a], mx[a + w]);
+        }
+        const float tile_max = mx[0] * p.scale_log2;
         float m_new = m_run, alpha = 1.f;
         if (tile_max > m_run + kRescaleThreshold) {
           m_new = tile_max;
           alpha = ex2(m_run - m_new);
         }
-        // p = 2^(s*c - m), row sum
+        // P = 2^(s*c - m): packed scale-subtract in fp32, rounded to bf16 pairs, MUFU ex2 on
+        // both halves at once; the row sum adds the same bf16 values P V will use.
+        const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2_pack(-m_new, -m_new);
+        const float neg_m = -m_new;
+        uint32_t pk[kTileK / 2];
         float rs[8];
 #pragma unroll
         for (int a = 0; a < 8; ++a) rs[a] = 0.f;
 #pragma unroll
-        for (int c = 0; c < kTileK; c += 8) {
-#pragma unroll
-          for (int a = 0; a < 8; ++a) {
-            const float e = ex2(fmaf(sv[c + a], p.scale_log2, -m_new));
-            sv[c + a] = e;
-            rs[a] += e;
-          }
+        for (int c = 0; c < kTileK / 2; ++c) {
+          float x0, x1;
+#if GCA_FMA2
+          f2_unpack(f2_fma(f2_pack(sv[2 * c], sv[2 * c + 1]), c2, nm2), x0, x1);
+#else
+          x0 = fmaf(sv[2 * c], p.scale_log2, neg_m);
+          x1 = fmaf(sv[2 * c + 1], p.scale_log2, neg_m);
+#endif
+#if GCA_EXP_BF16
+          pk[c] = ex2_bf2(pack_bf2(x0, x1));
+#if GCA_SUM_MIXED
+          add_bf2(rs[2 * (c & 3)], rs[2 * (c & 3) + 1], pk[c]);
+#else
+          rs[2 * (c & 3)] += __uint_as_float(pk[c] << 16);
+          rs[2 * (c & 3) + 1] += __uint_as_float(pk[c] & 0xffff0000u);
+#endif
+#else
+          const float e0 = ex2(x0), e1 = ex2(x1);
+          pk[c] = pack_bf2(e0, e1);
+          rs[2 * (c & 3)] += e0;
+          rs[2 * (c & 3) + 1] += e1;
+#endif
         }
+        (void)c2;
+        (void)nm2;
+        (void)neg_m;
         const float row_sum =
             ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
 
@@ -577,16 +653,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         l_run = l_run * alpha + row_sum;
         m_run = m_new;
-
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[kTileK / 4];
-#pragma unroll
-          for (int c = 0; c < kTileK / 4; ++c) {
-            pk[c] = pack_bf2(sv[64 * half + 2 * c], sv[64 * half + 2 * c + 1]);
-          }
-          tmem_st32(t_row + kColP + 32 * half, pk);
-        }
+        tmem_st32(t_row + kColP, pk);
+        tmem_st32(t_row + kColP + 32, pk + 32);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sh.p_full);
@@ -691,8 +759,11 @@ cudaError_t attn_prepare(int* ctas_per_sm) {
   int n = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel, kThreads, kSmemBytes);
   if (e != cudaSuccess) return e;
-  // Two CTAs share the SM's 512 TMEM columns (256 each); never more.
-  *ctas_per_sm = n < 1 ? 1 : (n > 2 ? 2 : n);
+  // Registers and shared memory admit two CTAs per SM and the two share the SM's 512 TMEM
+  // columns (256 each); the occupancy query ignores the shared-memory carveout, so it is only
+  // a lower bound here.
+  (void)n;
+  *ctas_per_sm = 2;
   return cudaSuccess;
 }
 
