@@ -35,12 +35,18 @@
 
 #include "gca_internal.h"
 
-// Softmax arithmetic options (defaults are the measured best on B200):
-//   GCA_EXP_BF16  1: P = ex2.bf16x2(bf16(s*c - m)) (two exponentials per MUFU issue);
-//                 0: fp32 ex2 per element, then rounded to bf16 pairs.
-//   GCA_FMA2      1: scale-subtract with packed f32x2 FMA; 0: scalar FMA.
-//   GCA_SUM_MIXED 1: row sum with mixed-precision bf16 -> fp32 adds; 0: plain fp32 adds.
-//   GCA_MAX_CHAINS independent 3-input max chains (4 or 8).
+// Softmax arithmetic options. The defaults are the fastest measured on B200 at head_dim 64:
+// fp32 ex2 (MUFU, 16/clk/SM) beats ex2.bf16x2 there because converting its input to bf16x2
+// shares a unit with it, and packed f32x2 arithmetic saves nothing once register pairs have
+// to be formed.
+//   GCA_EXP_BF16   1: P = ex2.bf16x2(bf16(s*c - m)); 0: fp32 ex2 per element, rounded to bf16.
+//   GCA_FMA2       1: scale-subtract with packed f32x2 FMA; 0: scalar FMA.
+//   GCA_SUM_MIXED  1: row sum with mixed-precision bf16 -> fp32 adds (bf16 path only).
+//   GCA_MAX_CHAINS independent 3-input max chains.
+//   GCA_STAGED     1: scale-subtract, exponentials and pack + sum run as separate passes over
+//                  the row, so independent MUFU operations issue back to back.
+//   GCA_SLEEP_WAIT 1: barrier waits suspend the thread in hardware (try_wait with a suspend
+//                  time hint) instead of spinning on issue slots.
 #ifndef GCA_EXP_BF16
 #define GCA_EXP_BF16 0
 #endif
@@ -51,7 +57,13 @@
 #define GCA_SUM_MIXED 1
 #endif
 #ifndef GCA_MAX_CHAINS
-#define GCA_MAX_CHAINS 4
+#define GCA_MAX_CHAINS 8
+#endif
+#ifndef GCA_STAGED
+#define GCA_STAGED 1
+#endif
+#ifndef GCA_SLEEP_WAIT
+#define GCA_SLEEP_WAIT 1
 #endif
 
 namespace gca {
@@ -121,12 +133,21 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
+#if GCA_SLEEP_WAIT
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(1000000u)
+      : "memory");
+#else
   asm volatile(
       "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_addr(bar)), "r"(parity)
       : "memory");
+#endif
   return ok != 0;
 }
 
@@ -138,7 +159,7 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, Share
   const uint64_t t0 = global_timer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0u) {
+    if (GCA_SLEEP_WAIT || (i & 63u) == 0u) {
       if (!drain && sh->abort_flag) return false;
       if (global_timer() - t0 > kWaitNs) {
         sh->abort_flag = 1;
@@ -596,8 +617,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           m_new = tile_max;
           alpha = ex2(m_run - m_new);
         }
-        // P = 2^(s*c - m): packed scale-subtract in fp32, rounded to bf16 pairs, MUFU ex2 on
-        // both halves at once; the row sum adds the same bf16 values P V will use.
+        // P = 2^(s*c - m), rounded to bf16 pairs for P V; the row sum accumulates the fp32
+        // values (the bf16 path sums the rounded values instead).
         const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
         const uint64_t nm2 = f2_pack(-m_new, -m_new);
         const float neg_m = -m_new;
@@ -605,6 +626,25 @@ __global__ void __launch_bounds__(kThreads, 2)
         float rs[8];
 #pragma unroll
         for (int a = 0; a < 8; ++a) rs[a] = 0.f;
+#if GCA_STAGED
+#pragma unroll
+        for (int e = 0; e < kTileK; ++e) sv[e] = fmaf(sv[e], p.scale_log2, neg_m);
+#if GCA_EXP_BF16
+#pragma unroll
+        for (int c = 0; c < kTileK / 2; ++c) pk[c] = ex2_bf2(pack_bf2(sv[2 * c], sv[2 * c + 1]));
+#pragma unroll
+        for (int c = 0; c < kTileK / 2; ++c) add_bf2(rs[2 * (c & 3)], rs[2 * (c & 3) + 1], pk[c]);
+#else
+#pragma unroll
+        for (int e = 0; e < kTileK; ++e) sv[e] = ex2(sv[e]);
+#pragma unroll
+        for (int c = 0; c < kTileK / 2; ++c) {
+          pk[c] = pack_bf2(sv[2 * c], sv[2 * c + 1]);
+          rs[2 * (c & 3)] += sv[2 * c];
+          rs[2 * (c & 3) + 1] += sv[2 * c + 1];
+        }
+#endif
+#else
 #pragma unroll
         for (int c = 0; c < kTileK / 2; ++c) {
           float x0, x1;
@@ -629,6 +669,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           rs[2 * (c & 3) + 1] += e1;
 #endif
         }
+#endif
         (void)c2;
         (void)nm2;
         (void)neg_m;
@@ -704,9 +745,12 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // Merges the partial records of every split unit: weights 2^(m_s - M), M = max_s m_s.
-__global__ void __launch_bounds__(kTileQ) combine_kernel(const AttnParams p) {
+// Two threads per query row, 32 output columns each.
+constexpr int kCombineThreads = 2 * kTileQ;
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const AttnParams p) {
   const int u = blockIdx.x;
-  const int r = threadIdx.x;
+  const int r = threadIdx.x >> 1;
+  const int half = threadIdx.x & 1;
   const int64_t first = (int64_t)u * p.n_tiles;
   const int64_t c0 = cta_of_step(first, p.total, p.grid);
   const int64_t c1 = cta_of_step(first + p.n_tiles - 1, p.total, p.grid);
@@ -716,18 +760,19 @@ __global__ void __launch_bounds__(kTileQ) combine_kernel(const AttnParams p) {
   if (qi >= p.T) return;
   float M = -INFINITY;
   for (int64_t c = c0; c <= c1; ++c) M = fmaxf(M, p.part_ml[(c + u) * kTileQ + r].x);
-  float acc[kHeadDim];
+  float acc[32];
 #pragma unroll
-  for (int a = 0; a < kHeadDim; ++a) acc[a] = 0.f;
+  for (int a = 0; a < 32; ++a) acc[a] = 0.f;
   float L = 0.f;
   for (int64_t c = c0; c <= c1; ++c) {
     const float2 ml = p.part_ml[(c + u) * kTileQ + r];
     const float w = ex2(ml.x - M);
     L += w * ml.y;
-    const float4* src = reinterpret_cast<const float4*>(p.part_o + ((c + u) * kTileQ + r) * kHeadDim);
+    const float4* src = reinterpret_cast<const float4*>(
+        p.part_o + ((c + u) * kTileQ + r) * kHeadDim + 32 * half);
 #pragma unroll
-    for (int a = 0; a < kHeadDim / 4; ++a) {
-      const float4 v = src[a];
+    for (int a = 0; a < 8; ++a) {
+      const float4 v = __ldcg(src + a);
       acc[4 * a] += w * v.x;
       acc[4 * a + 1] += w * v.y;
       acc[4 * a + 2] += w * v.z;
@@ -735,9 +780,9 @@ __global__ void __launch_bounds__(kTileQ) combine_kernel(const AttnParams p) {
     }
   }
   const float inv = 1.f / L;
-  uint4* dst = p.out + ((int64_t)qi * p.H + h) * 8;
+  uint4* dst = p.out + ((int64_t)qi * p.H + h) * 8 + 4 * half;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < 4; ++c) {
     uint4 w;
     w.x = pack_bf2(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
     w.y = pack_bf2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
@@ -774,7 +819,7 @@ cudaError_t launch_attn(const CUtensorMap& tk, const CUtensorMap& tv, const Attn
 }
 
 cudaError_t launch_combine(const AttnParams& p, cudaStream_t s) {
-  combine_kernel<<<p.units, kTileQ, 0, s>>>(p);
+  combine_kernel<<<p.units, kCombineThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
