@@ -146,6 +146,22 @@ gca_status gca_append_frame(gca_cache* cache, int64_t frame_idx, const void* q, 
 gca_status gca_attend(gca_cache* cache, int64_t frame_idx, const void* q_rot, void* out,
                       void* stream);
 
+/* The same attention as gca_attend, for callers that may not allocate device memory while
+ * they run: a process that budgets all GPU memory when it starts and treats any later
+ * cudaMalloc as a failure, a plugin whose host application owns the device allocator, or a
+ * latency-critical loop where a cudaMalloc (which can synchronise the device) is not allowed.
+ * It allocates nothing. Its scratch -- the split-KV partial records -- lives in a 16 MiB array
+ * inside this library, which every GPU that loads the library holds until the process exits.
+ * The first call on a device looks up that array's device address (cudaGetSymbolAddress) with
+ * the device current; make that first call before any stream capture. All calls share the one
+ * array and it keeps the last call's contents (every slot read is written earlier in the same
+ * call): calls whose kernels overlap on the GPU race on it, so order them (one stream, or
+ * events). Returns GCA_ERR_UNSUPPORTED when a frame needs more partial records than the array
+ * holds, i.e. when num_heads * ceil(T / 128) >= 496; other errors as gca_attend.
+ * The web pages have no counterpart of this entry point; it is an addition of this library. */
+gca_status gca_attend_noalloc(gca_cache* cache, int64_t frame_idx, const void* q_rot, void* out,
+                              void* stream);
+
 /* Restores the state of a new stream (pages' clean_kv_cache): free list back to its initial
  * order, counters to zero, device error word cleared. Enqueued on `stream`. */
 gca_status gca_reset(gca_cache* cache, void* stream);

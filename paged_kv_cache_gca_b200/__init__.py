@@ -17,7 +17,7 @@ __all__ = [
     "GcaError", "GcaConfig", "GcaState", "GcaAttendInfo", "lib", "library_path",
     "gca_validate_config", "gca_workspace_bytes", "gca_cache_create", "gca_append_frame",
     "gca_attend", "gca_reset", "gca_cache_destroy", "gca_check", "gca_get_state",
-    "gca_last_attend_info", "gca_status_string", "GcaCache", "config_for",
+    "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc", "GcaCache", "config_for",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -78,7 +78,7 @@ class GcaAttendInfo(ctypes.Structure):
 EXPORTED_SYMBOLS = (
     "gca_validate_config", "gca_workspace_bytes", "gca_cache_create", "gca_append_frame",
     "gca_attend", "gca_reset", "gca_cache_destroy", "gca_check", "gca_get_state",
-    "gca_last_attend_info", "gca_status_string",
+    "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc",
 )
 
 _lib = None
@@ -108,6 +108,7 @@ def lib():
         "gca_get_state": (I32, [VP, P(GcaState)]),
         "gca_last_attend_info": (I32, [VP, P(GcaAttendInfo)]),
         "gca_status_string": (ctypes.c_char_p, [I32]),
+        "gca_attend_noalloc": (I32, [VP, I64, VP, VP, VP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -149,6 +150,12 @@ def gca_append_frame(handle, frame_idx, q_ptr, k_ptr, v_ptr, q_rot_ptr, stream) 
 
 def gca_attend(handle, frame_idx, q_rot_ptr, out_ptr, stream) -> None:
     _ok(lib().gca_attend(handle, frame_idx, q_rot_ptr, out_ptr, stream), "gca_attend")
+
+
+def gca_attend_noalloc(handle, frame_idx, q_rot_ptr, out_ptr, stream) -> None:
+    """gca_attend with its scratch in the library's fixed device array (no allocation)."""
+    _ok(lib().gca_attend_noalloc(handle, frame_idx, q_rot_ptr, out_ptr, stream),
+        "gca_attend_noalloc")
 
 
 def gca_reset(handle, stream) -> None:

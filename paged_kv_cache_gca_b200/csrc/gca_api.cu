@@ -12,26 +12,6 @@
 
 #include "gca_internal.h"
 
-struct gca_cache {
-  gca_config cfg;
-  gca::Layout lay;
-  char* ws;
-  int device;
-  int sms;
-  int ctas_per_sm;
-  int64_t frames;
-  int64_t free_head;
-  int64_t free_tail;
-  int64_t traj_len;
-  int32_t traj_pages;
-  int32_t n_kept;
-  int32_t kept[gca::kMaxKeep];
-  uint32_t dev_err;
-  CUtensorMap tm_k;
-  CUtensorMap tm_v;
-  gca_attend_info last;
-};
-
 namespace gca {
 
 namespace {
