@@ -156,8 +156,9 @@ gca_status gca_attend(gca_cache* cache, int64_t frame_idx, const void* q_rot, vo
  * the device current; make that first call before any stream capture. All calls share the one
  * array and it keeps the last call's contents (every slot read is written earlier in the same
  * call): calls whose kernels overlap on the GPU race on it, so order them (one stream, or
- * events). Returns GCA_ERR_UNSUPPORTED when a frame needs more partial records than the array
- * holds, i.e. when num_heads * ceil(T / 128) >= 496; other errors as gca_attend.
+ * events). The array holds 496 partial records of 128 query rows; a launch over num_heads *
+ * ceil(T / 256) query-tile pairs needs two per pair and two per CTA, so this returns
+ * GCA_ERR_UNSUPPORTED when num_heads * ceil(T / 256) >= 248; other errors as gca_attend.
  * The web pages have no counterpart of this entry point; it is an addition of this library. */
 gca_status gca_attend_noalloc(gca_cache* cache, int64_t frame_idx, const void* q_rot, void* out,
                               void* stream);

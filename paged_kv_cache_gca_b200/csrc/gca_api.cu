@@ -128,12 +128,67 @@ bool compute_layout(const gca_config& c, Layout* L) {
   L->slot_map = take(4 * (size_t)T);
   L->kept = take(4 * (size_t)kMaxKeep);
   L->rope_t = take(8 * (size_t)c.max_frames * L->nt);
-  L->rope_y = take(8 * (size_t)(c.grid_h + 1) * L->ny);
-  L->rope_x = take(8 * (size_t)(c.grid_w + 1) * L->nx);
+  L->rope_tok = take(8 * (size_t)T * (L->ny + L->nx));
   L->err = take(4);
   L->part_o = take(4 * (size_t)L->part_slots * kTileQ * kHeadDim);
   L->part_ml = take(8 * (size_t)L->part_slots * kTileQ);
   L->total = align_up(off, kAlign);
+  return true;
+}
+
+bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams* p,
+                    bool* split, int64_t* visible_keys) {
+  const Layout& L = c->lay;
+  const gca_config& cf = c->cfg;
+  int64_t na_frames, w0, nwf;
+  if (t < cf.anchor_frames) {
+    na_frames = t + 1;
+    w0 = 0;
+    nwf = 0;
+  } else {
+    na_frames = cf.anchor_frames;
+    w0 = std::max<int64_t>(cf.anchor_frames, t - cf.window_frames + 1);
+    nwf = t - w0 + 1;
+  }
+  std::memset(p, 0, sizeof(*p));
+  p->frame_pages = reinterpret_cast<const int32_t*>(c->ws + L.frame_pages);
+  p->traj_pages = reinterpret_cast<const int32_t*>(c->ws + L.traj_pages);
+  p->err = reinterpret_cast<uint32_t*>(c->ws + L.err);
+  p->T = L.T;
+  p->H = cf.num_heads;
+  p->ppf = L.ppf;
+  p->last_len = L.last_len;
+  p->num_pages = cf.num_pages;
+  p->na_pages = (int32_t)(na_frames * L.ppf);
+  p->win_base = (int32_t)(w0 * L.ppf);
+  p->nw_pages = (int32_t)(nwf * L.ppf);
+  p->n_traj_pages = c->traj_pages;
+  p->traj_tail_len =
+      c->traj_pages > 0 ? (int32_t)(c->traj_len - (int64_t)(c->traj_pages - 1) * kPageSize) : 0;
+  p->n_lp = p->na_pages + p->nw_pages + p->n_traj_pages;
+  p->n_tiles = (p->n_lp + kPagesPerTile - 1) / kPagesPerTile;
+  p->n_qt = L.n_qt;
+  p->units = cf.num_heads * L.n_qt;
+  p->n_pairs = (L.n_qt + 1) / 2;
+  p->units2 = cf.num_heads * p->n_pairs;
+  p->total = (int64_t)p->units2 * p->n_tiles;
+  int64_t gmax = std::min<int64_t>(kMaxGrid, (int64_t)c->sms * c->ctas_per_sm);
+  gmax = std::min<int64_t>(gmax, max_slots / 2 - p->units2);  // partial slots must fit
+  if (gmax < 1) return false;
+  int64_t g = (p->total + kMinStepsPerCta - 1) / kMinStepsPerCta;
+  g = std::max<int64_t>(g, std::min<int64_t>(p->units2, gmax));
+  g = std::min<int64_t>(g, gmax);
+  g = std::min<int64_t>(g, p->total);
+  p->grid = (int32_t)g;
+  p->scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)cf.head_dim));
+  bool sp = false;
+  for (int u = 0; u < p->units2 && !sp; ++u) {
+    const int64_t first = (int64_t)u * p->n_tiles;
+    sp = cta_of_step(first, p->total, p->grid) !=
+         cta_of_step(first + p->n_tiles - 1, p->total, p->grid);
+  }
+  *split = sp;
+  *visible_keys = (na_frames + nwf) * L.T + c->traj_len;
   return true;
 }
 
@@ -240,13 +295,14 @@ gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t w
     ip.user_free = dev_initial_free_list;
     ip.kept = at<int32_t>(c, L.kept);
     ip.rope_t = at<float2>(c, L.rope_t);
-    ip.rope_y = at<float2>(c, L.rope_y);
-    ip.rope_x = at<float2>(c, L.rope_x);
+    ip.rope_tok = at<float2>(c, L.rope_tok);
     ip.err = at<uint32_t>(c, L.err);
     ip.num_pages = cfg->num_pages;
     ip.max_frames = cfg->max_frames;
     ip.grid_h = cfg->grid_h;
     ip.grid_w = cfg->grid_w;
+    ip.num_special = cfg->num_special;
+    ip.T = L.T;
     ip.nt = L.nt;
     ip.ny = L.ny;
     ip.nx = L.nx;
@@ -296,22 +352,18 @@ gca_status gca_append_frame(gca_cache* c, int64_t t, const void* q, const void* 
   p.slot_map = at<int32_t>(c, L.slot_map);
   p.kept = at<int32_t>(c, L.kept);
   p.rope_t = at<float2>(c, L.rope_t);
-  p.rope_y = at<float2>(c, L.rope_y);
-  p.rope_x = at<float2>(c, L.rope_x);
+  p.rope_tok = at<float2>(c, L.rope_tok);
   p.err = at<uint32_t>(c, L.err);
   p.t = t;
-  p.free_head = c->free_head;
-  p.free_tail = c->free_tail;
   p.traj_len = c->traj_len;
+  p.head_pos = (int32_t)(c->free_head % cf.num_pages);
+  p.tail_pos = (int32_t)(c->free_tail % cf.num_pages);
   p.T = L.T;
   p.H = cf.num_heads;
-  p.S = cf.num_special;
-  p.grid_w = cf.grid_w;
   p.ppf = L.ppf;
   p.num_pages = cf.num_pages;
   p.nt = L.nt;
-  p.ny = L.ny;
-  p.nx = L.nx;
+  p.nyx = L.ny + L.nx;
   p.evict_frame = evict ? (int32_t)e : -1;
   p.K = K;
   p.traj_pages_before = c->traj_pages;
@@ -321,13 +373,13 @@ gca_status gca_append_frame(gca_cache* c, int64_t t, const void* q, const void* 
                      ? (int32_t)(kPageSize - end_pos % kPageSize)
                      : 0;
   const int64_t per_tok = (int64_t)cf.num_heads * 8;
-  p.n_tok_items = (int64_t)L.ppf * kPageSize * per_tok;
+  p.tok_per_block = std::max<int32_t>(1, 256 / (int32_t)per_tok);
+  p.n_tok_blocks = (int32_t)((L.ppf * kPageSize + p.tok_per_block - 1) / p.tok_per_block);
   p.n_evict_items = (int64_t)K * per_tok;
   p.n_zero_items = (int64_t)p.zero_slots * per_tok;
   p.n_push_items = evict ? L.ppf : 0;
   p.n_traj_items = n_pop_traj;
-  p.n_items = p.n_tok_items + p.n_evict_items + p.n_zero_items + p.n_push_items +
-              p.n_traj_items;
+  p.n_aux_items = p.n_evict_items + p.n_zero_items + p.n_push_items + p.n_traj_items;
   if (launch_append(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GCA_ERR_CUDA;
 
   c->free_head += L.ppf + n_pop_traj;
@@ -343,63 +395,21 @@ gca_status gca_attend(gca_cache* c, int64_t t, const void* q_rot, void* out, voi
   if (c->frames == 0 || t != c->frames - 1) return GCA_ERR_FRAME_ORDER;
   if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;
   const Layout& L = c->lay;
-  const gca_config& cf = c->cfg;
-  int64_t na_frames, w0, nwf;
-  if (t < cf.anchor_frames) {
-    na_frames = t + 1;
-    w0 = 0;
-    nwf = 0;
-  } else {
-    na_frames = cf.anchor_frames;
-    w0 = std::max<int64_t>(cf.anchor_frames, t - cf.window_frames + 1);
-    nwf = t - w0 + 1;
-  }
   AttnParams p;
-  std::memset(&p, 0, sizeof(p));
+  bool split = false;
+  int64_t nk = 0;
+  if (!plan_attention(c, t, L.part_slots, &p, &split, &nk)) return GCA_ERR_UNSUPPORTED;
   p.q = static_cast<const uint4*>(q_rot);
   p.out = static_cast<uint4*>(out);
   p.part_o = at<float>(c, L.part_o);
   p.part_ml = at<float2>(c, L.part_ml);
-  p.frame_pages = at<int32_t>(c, L.frame_pages);
-  p.traj_pages = at<int32_t>(c, L.traj_pages);
-  p.err = at<uint32_t>(c, L.err);
-  p.T = L.T;
-  p.H = cf.num_heads;
-  p.ppf = L.ppf;
-  p.last_len = L.last_len;
-  p.num_pages = cf.num_pages;
-  p.na_pages = (int32_t)(na_frames * L.ppf);
-  p.win_base = (int32_t)(w0 * L.ppf);
-  p.nw_pages = (int32_t)(nwf * L.ppf);
-  p.n_traj_pages = c->traj_pages;
-  p.traj_tail_len =
-      c->traj_pages > 0 ? (int32_t)(c->traj_len - (int64_t)(c->traj_pages - 1) * kPageSize) : 0;
-  p.n_lp = p.na_pages + p.nw_pages + p.n_traj_pages;
-  p.n_tiles = (p.n_lp + kPagesPerTile - 1) / kPagesPerTile;
-  p.n_qt = L.n_qt;
-  p.units = cf.num_heads * L.n_qt;
-  p.total = (int64_t)p.units * p.n_tiles;
-  const int64_t gmax = std::min<int64_t>(kMaxGrid, (int64_t)c->sms * c->ctas_per_sm);
-  int64_t g = (p.total + kMinStepsPerCta - 1) / kMinStepsPerCta;
-  g = std::max<int64_t>(g, std::min<int64_t>(p.units, gmax));
-  g = std::min<int64_t>(g, gmax);
-  g = std::min<int64_t>(g, p.total);
-  p.grid = (int32_t)g;
-  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)cf.head_dim));
-
-  bool split = false;
-  for (int u = 0; u < p.units && !split; ++u) {
-    const int64_t first = (int64_t)u * p.n_tiles;
-    split = cta_of_step(first, p.total, p.grid) !=
-            cta_of_step(first + p.n_tiles - 1, p.total, p.grid);
-  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (launch_attn(c->tm_k, c->tm_v, p, s) != cudaSuccess) return GCA_ERR_CUDA;
   if (split && launch_combine(p, s) != cudaSuccess) return GCA_ERR_CUDA;
 
   gca_attend_info& inf = c->last;
   inf.frame_idx = t;
-  inf.visible_keys = (na_frames + nwf) * L.T + c->traj_len;
+  inf.visible_keys = nk;
   inf.logical_pages = p.n_lp;
   inf.kv_tiles = p.n_tiles;
   inf.query_tiles = L.n_qt;

@@ -28,10 +28,6 @@ constexpr int kThreads = 256;
 
 __device__ __forceinline__ void set_err(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
 
-__device__ __forceinline__ int ring_at(const int32_t* ring, int64_t pos, int32_t n) {
-  return ring[pos % n];
-}
-
 // ------------------------------------------------------------------------------- init
 
 __global__ void init_kernel(const InitParams p) {
@@ -49,25 +45,43 @@ __global__ void init_kernel(const InitParams p) {
     }
   }
   for (int64_t i = tid; i < p.keep; i += stride) p.kept[i] = p.kept_host[i];
-  // RoPE tables in fp64, stored as fp32 (cos, sin): angle = pos * base^(-2j/d)
+  // RoPE tables in fp64, stored as fp32 (cos, sin): pair j of a band of width d turns by
+  // pos * base^(-2j/d). Time band per frame; the two spatial bands per token (camera/register
+  // tokens at (y, x) = (0, 0), the patch at row r, column c at (r+1, c+1)).
   const int64_t n_t = (int64_t)p.max_frames * p.nt;
-  const int64_t n_y = (int64_t)(p.grid_h + 1) * p.ny;
-  const int64_t n_x = (int64_t)(p.grid_w + 1) * p.nx;
-  for (int64_t i = tid; i < n_t + n_y + n_x; i += stride) {
+  const int nyx = p.ny + p.nx;
+  const int64_t n_s = (int64_t)p.T * nyx;
+  for (int64_t i = tid; i < n_t + n_s; i += stride) {
     int64_t pos, j;
     int d;
     float2* dst;
     if (i < n_t) {
-      pos = i / p.nt; j = i % p.nt; d = 2 * p.nt; dst = p.rope_t + i;
-    } else if (i < n_t + n_y) {
-      int64_t r = i - n_t;
-      pos = r / p.ny; j = r % p.ny; d = 2 * p.ny; dst = p.rope_y + r;
+      pos = i / p.nt;
+      j = i % p.nt;
+      d = 2 * p.nt;
+      dst = p.rope_t + i;
     } else {
-      int64_t r = i - n_t - n_y;
-      pos = r / p.nx; j = r % p.nx; d = 2 * p.nx; dst = p.rope_x + r;
+      const int64_t r = i - n_t;
+      const int64_t tok = r / nyx;
+      const int64_t pr = r % nyx;  // pair index within the spatial bands
+      int64_t y = 0, x = 0;
+      if (tok >= p.num_special) {
+        y = (tok - p.num_special) / p.grid_w + 1;
+        x = (tok - p.num_special) % p.grid_w + 1;
+      }
+      if (pr < p.ny) {
+        pos = y;
+        j = pr;
+        d = 2 * p.ny;
+      } else {
+        pos = x;
+        j = pr - p.ny;
+        d = 2 * p.nx;
+      }
+      dst = p.rope_tok + r;
     }
-    double inv_freq = pow(p.base, -2.0 * (double)j / (double)d);
-    double ang = (double)pos * inv_freq;
+    const double inv_freq = pow(p.base, -2.0 * (double)j / (double)d);
+    const double ang = (double)pos * inv_freq;
     double sn, cs;
     sincos(ang, &sn, &cs);
     *dst = make_float2((float)cs, (float)sn);
@@ -104,22 +118,20 @@ __device__ __forceinline__ uint32_t rotate_word(uint32_t w, float2 cs) {
   return pack_bf2(ra, rb);
 }
 
-__global__ void __launch_bounds__(kThreads) append_kernel(const AppendParams p) {
-  const int64_t idx = blockIdx.x * (int64_t)kThreads + threadIdx.x;
-  if (idx >= p.n_items) return;
-  const int H = p.H;
-  const int64_t e_tok = p.n_tok_items;
-  const int64_t e_ev = e_tok + p.n_evict_items;
-  const int64_t e_zero = e_ev + p.n_zero_items;
-  const int64_t e_push = e_zero + p.n_push_items;
+__device__ __forceinline__ int wrap(int pos, int n) { return pos >= n ? pos - n : pos; }
 
-  if (idx < e_tok) {
-    // ---- a1 + a2: one 16-byte chunk (8 dims) of one (token, head)
-    const int c = (int)(idx & 7);
-    const int64_t th = idx >> 3;
-    const int h = (int)(th % H);
-    const int i = (int)(th / H);
-    const int page = ring_at(p.free_ring, p.free_head + i / kPageSize, p.num_pages);
+// Token part: block (8 chunks, H heads, tok_per_block tokens); one thread = one 16-byte chunk
+// (8 dims) of one (token, head). Auxiliary part (blocks after n_tok_blocks): eviction copies,
+// zero fill of a fresh trajectory page, free-list pushes, trajectory page records.
+__global__ void __launch_bounds__(1024) append_kernel(const AppendParams p) {
+  const int H = p.H;
+  if (blockIdx.x < (unsigned)p.n_tok_blocks) {
+    // ---- a1 + a2
+    const int c = threadIdx.x;
+    const int h = threadIdx.y;
+    const int i = blockIdx.x * p.tok_per_block + threadIdx.z;
+    if (i >= p.ppf * kPageSize) return;
+    const int page = p.free_ring[wrap(p.head_pos + i / kPageSize, p.num_pages)];
     if (page < 0 || page >= p.num_pages) {
       set_err(p.err, GCA_DEVERR_PAGE_RANGE);
       return;
@@ -139,24 +151,11 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const AppendParams p) 
     const uint4 qv = p.q[src];
     const uint4 kv = p.k[src];
     const uint4 vv = p.v[src];
-    // positions: camera/register tokens at (t, 0, 0); patch (r, c) at (t, r+1, c+1)
-    int ypos = 0, xpos = 0;
-    if (i >= p.S) {
-      const int pidx = i - p.S;
-      ypos = pidx / p.grid_w + 1;
-      xpos = pidx % p.grid_w + 1;
-    }
     float2 cs[4];
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const int j = 4 * c + w;  // pair index within the head
-      if (j < p.nt) {
-        cs[w] = p.rope_t[p.t * p.nt + j];
-      } else if (j < p.nt + p.ny) {
-        cs[w] = p.rope_y[ypos * p.ny + (j - p.nt)];
-      } else {
-        cs[w] = p.rope_x[xpos * p.nx + (j - p.nt - p.ny)];
-      }
+      cs[w] = j < p.nt ? p.rope_t[p.t * p.nt + j] : p.rope_tok[(int64_t)i * p.nyx + (j - p.nt)];
     }
     uint4 qr, kr;
     qr.x = rotate_word(qv.x, cs[0]);
@@ -173,11 +172,19 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const AppendParams p) 
     return;
   }
 
+  const int block_threads = 8 * H * p.tok_per_block;
+  const int lin = threadIdx.x + 8 * (threadIdx.y + H * threadIdx.z);
+  const int64_t idx = (int64_t)(blockIdx.x - p.n_tok_blocks) * block_threads + lin;
+  if (idx >= p.n_aux_items) return;
+  const int64_t e_ev = p.n_evict_items;
+  const int64_t e_zero = e_ev + p.n_zero_items;
+  const int64_t e_push = e_zero + p.n_push_items;
+  const int first_new = wrap(p.head_pos + p.ppf, p.num_pages);  // first trajectory pop
+
   if (idx < e_ev) {
     // ---- a3: copy kept token j of the evicted frame to trajectory position traj_len + j
-    const int64_t r = idx - e_tok;
-    const int c = (int)(r & 7);
-    const int64_t th = r >> 3;
+    const int c = (int)(idx & 7);
+    const int64_t th = idx >> 3;
     const int h = (int)(th % H);
     const int j = (int)(th / H);
     const int tok = p.kept[j];
@@ -187,7 +194,7 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const AppendParams p) 
     const int dst_page =
         tp < p.traj_pages_before
             ? p.traj_pages[tp]
-            : ring_at(p.free_ring, p.free_head + p.ppf + (tp - p.traj_pages_before), p.num_pages);
+            : p.free_ring[wrap(first_new + (int)(tp - p.traj_pages_before), p.num_pages)];
     if (src_page < 0 || src_page >= p.num_pages || dst_page < 0 || dst_page >= p.num_pages) {
       set_err(p.err, GCA_DEVERR_PAGE_RANGE);
       return;
@@ -209,7 +216,7 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const AppendParams p) 
     const int64_t pos = p.traj_len + p.K + z;
     const int64_t tp = pos / kPageSize;
     const int page =
-        ring_at(p.free_ring, p.free_head + p.ppf + (tp - p.traj_pages_before), p.num_pages);
+        p.free_ring[wrap(first_new + (int)(tp - p.traj_pages_before), p.num_pages)];
     if (page < 0 || page >= p.num_pages) {
       set_err(p.err, GCA_DEVERR_PAGE_RANGE);
       return;
@@ -223,23 +230,21 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const AppendParams p) 
   if (idx < e_push) {
     // ---- push the evicted frame's pages to the free-list tail, in row order
     const int k = (int)(idx - e_zero);
-    p.free_ring[(p.free_tail + k) % p.num_pages] =
+    p.free_ring[wrap(p.tail_pos + k, p.num_pages)] =
         p.frame_pages[(int64_t)p.evict_frame * p.ppf + k];
     return;
   }
 
   // ---- record the trajectory pages popped by this step
   const int k = (int)(idx - e_push);
-  p.traj_pages[p.traj_pages_before + k] =
-      ring_at(p.free_ring, p.free_head + p.ppf + k, p.num_pages);
+  p.traj_pages[p.traj_pages_before + k] = p.free_ring[wrap(first_new + k, p.num_pages)];
 }
 
 }  // namespace
 
 cudaError_t launch_init(const InitParams& p, cudaStream_t s) {
   int64_t work = p.num_pages;
-  int64_t rope = (int64_t)p.max_frames * p.nt + (int64_t)(p.grid_h + 1) * p.ny +
-                 (int64_t)(p.grid_w + 1) * p.nx;
+  const int64_t rope = (int64_t)p.max_frames * p.nt + (int64_t)p.T * (p.ny + p.nx);
   if (rope > work) work = rope;
   int64_t blocks = (work + kThreads - 1) / kThreads;
   if (blocks > 4096) blocks = 4096;
@@ -260,8 +265,10 @@ cudaError_t launch_reset(int32_t* free_ring, const int32_t* init_free, uint32_t*
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
-  const int64_t blocks = (p.n_items + kThreads - 1) / kThreads;
-  append_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(p);
+  const int64_t block_threads = 8LL * p.H * p.tok_per_block;
+  const int64_t aux_blocks = (p.n_aux_items + block_threads - 1) / block_threads;
+  const dim3 block(8, p.H, p.tok_per_block);
+  append_kernel<<<(unsigned)(p.n_tok_blocks + aux_blocks), block, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -13,89 +13,122 @@
 // the page table. A 128-key tile is 8 pages; each page of one head is a contiguous 2 KB block
 // [16 slots][64 dims] bf16 that TMA copies into shared memory with the 128-byte swizzle.
 //
-// Work split: a (head, 128-query tile) pair is a unit; the flattened (unit, key tile) steps are
-// cut into `grid` equal ranges, one per CTA. A unit that spans several CTAs leaves partial
-// (O, row max, row sum) records that a combine kernel merges with log-sum-exp weights.
+// Work split: a CTA works on two 128-query tiles of one head at once (they see the same keys,
+// so every K/V tile is fetched once for both); a (head, tile pair) is a work unit. The flattened
+// (unit, key tile) steps are cut into `grid` equal ranges, one per CTA (one CTA per SM). A unit
+// that spans several CTAs leaves partial (O, row max, row sum) records per query tile that a
+// combine kernel merges with log-sum-exp weights.
 //
-// CTA roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r). Loads Q into swizzled shared
-//              memory; per key tile reads S from TMEM, masks, does the online softmax in fp32
-//              with exp2, writes P (bf16) to TMEM, and rescales the O accumulator in TMEM only
-//              when the row max grows by more than 2^8 (lazy rescale). Epilogue writes O / l.
-//   warp 4     TMA producer: resolves the tile's 8 page ids and issues 16 page copies (K, V)
-//              per tile into a 3-stage ring.
-//   warp 5     MMA issuer (one thread): S = Q K^T (A, B from shared memory) into TMEM, then
-//              O += P V with P read from TMEM (A operand in tensor memory) and V from shared
-//              memory (MN-major). S of tile j+1 is issued before P V of tile j so the tensor
-//              core works while the softmax threads do.
-// TMEM (256 columns): S fp32 [0,128), P bf16x2 [128,192), O fp32 [192,256).
+// CTA roles (352 threads):
+//   warps 0-3, 4-7  softmax warpgroup of query tile 0 / 1: thread r owns query row r (TMEM lane
+//              r). Loads its Q tile into swizzled shared memory; per key tile reads S from TMEM,
+//              masks unused page slots, takes the row max, then -- taking turns with the other
+//              warpgroup, because the exponentials are the bottleneck (MUFU) -- computes
+//              P = 2^(s*log2e/sqrt(D) - m), writes it to TMEM as bf16 and accumulates the row
+//              sum; O in TMEM is rescaled only when the row max grows by more than 2^8.
+//   warp 8     TMA producer: resolves the tile's 8 page ids and issues 16 page copies (K, V)
+//              per tile into 3-stage K and V rings.
+//   warps 9,10 MMA issuers, one per query tile (one thread issues only about one tcgen05.mma
+//              per 60 cycles): S = Q K^T (A, B from shared memory) into TMEM, then O += P V with
+//              P read from TMEM (A operand in tensor memory) and V from shared memory (MN-major).
+//              S of tile j+1 is issued as soon as S of tile j has been read.
+// TMEM (512 columns): per query tile q, q*256 + {S fp32 [0,128), P bf16x2 [128,192),
+// O fp32 [192,256)}.
 // Every wait is bounded in time; on expiry the kernel sets GCA_DEVERR_WAIT_TIMEOUT, drains its
 // own copies, frees TMEM and returns.
 #include <cuda_bf16.h>
 
 #include "gca_internal.h"
 
-// Softmax arithmetic options. The defaults are the fastest measured on B200 at head_dim 64:
-// fp32 ex2 (MUFU, 16/clk/SM) beats ex2.bf16x2 there because converting its input to bf16x2
-// shares a unit with it, and packed f32x2 arithmetic saves nothing once register pairs have
-// to be formed.
-//   GCA_EXP_BF16   1: P = ex2.bf16x2(bf16(s*c - m)); 0: fp32 ex2 per element, rounded to bf16.
-//   GCA_FMA2       1: scale-subtract with packed f32x2 FMA; 0: scalar FMA.
-//   GCA_SUM_MIXED  1: row sum with mixed-precision bf16 -> fp32 adds (bf16 path only).
-//   GCA_MAX_CHAINS independent 3-input max chains.
-//   GCA_STAGED     1: scale-subtract, exponentials and pack + sum run as separate passes over
-//                  the row, so independent MUFU operations issue back to back.
+// Build options (defaults are the fastest measured on B200 at head_dim 64):
+//   GCA_MAX_CHAINS independent 3-input max chains for the row max.
 //   GCA_SLEEP_WAIT 1: barrier waits suspend the thread in hardware (try_wait with a suspend
 //                  time hint) instead of spinning on issue slots.
-#ifndef GCA_EXP_BF16
-#define GCA_EXP_BF16 0
-#endif
-#ifndef GCA_FMA2
-#define GCA_FMA2 0
-#endif
-#ifndef GCA_SUM_MIXED
-#define GCA_SUM_MIXED 1
-#endif
 #ifndef GCA_MAX_CHAINS
 #define GCA_MAX_CHAINS 8
-#endif
-#ifndef GCA_STAGED
-#define GCA_STAGED 1
 #endif
 #ifndef GCA_SLEEP_WAIT
 #define GCA_SLEEP_WAIT 1
 #endif
+//   GCA_TURN_SPIN  0: the exponential-turn wait sleeps in hardware; 1: it spins; n >= 2: it
+//                  spins with __nanosleep(n) between polls.
+//   GCA_TURN_EARLY the turn passes to the other warpgroup this many 32-column chunks before
+//                  this one's exponentials are done.
+//   GCA_TURNS      1: the two softmax warpgroups take turns for the exponentials; 0: both
+//                  compute them whenever their scores are ready.
+#ifndef GCA_TURNS
+#define GCA_TURNS 1
+#endif
+#ifndef GCA_TURN_SPIN
+#define GCA_TURN_SPIN 1
+#endif
+#ifndef GCA_TURN_EARLY
+#define GCA_TURN_EARLY 1
+#endif
+//   GCA_POLY_PAIRS of every 16 pairs of exponentials, this many are computed on the FMA pipe
+//                  with a cubic polynomial instead of MUFU (relieves the MUFU bottleneck).
+#ifndef GCA_POLY_PAIRS
+#define GCA_POLY_PAIRS 0
+#endif
+
+#ifndef GCA_TRACE
+#define GCA_TRACE 0
+#endif
 
 namespace gca {
 
+#if GCA_TRACE
+// Event timestamps (clock64) of the first tiles of CTAs 0 and 1, for pipeline studies; read
+// back with gca_debug_trace in builds with -DGCA_TRACE=1.
+__device__ long long g_trace[2][64][16];
+#define TRACE(slot, tile)                                                                   \
+  do {                                                                                      \
+    if (blockIdx.x < 2 && (tile) < 64) g_trace[blockIdx.x][(tile)][(slot)] = clock64();     \
+  } while (0)
+#else
+#define TRACE(slot, tile) \
+  do {                    \
+  } while (0)
+#endif
+
 namespace {
 
-constexpr int kStages = 3;
-constexpr int kThreads = 192;
-constexpr int kWarpTma = 4;
-constexpr int kWarpMma = 5;
+constexpr int kQPerCta = 2;        // query tiles per CTA (same head: they share every K/V tile)
+constexpr int kKStages = 3;        // K ring: a slot frees once both S = Q K^T are computed
+constexpr int kVStages = 3;        // V ring: a slot frees after both O += P V
+constexpr int kSoftmaxWarps = 4 * kQPerCta;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 1 + kQPerCta);  // + TMA warp + MMA warps
+constexpr int kWarpTma = kSoftmaxWarps;
+constexpr int kWarpMma0 = kSoftmaxWarps + 1;  // MMA warp of query tile q: kWarpMma0 + q
 constexpr uint32_t kTileBytes = kTileK * kHeadDim * 2;      // 16 KB
 constexpr uint32_t kPageBytes = kPageSize * kHeadDim * 2;    // 2 KB
-constexpr uint32_t kTmemCols = 256;
-// TMEM columns: S fp32 [0,128), P bf16x2 [128,192), O fp32 [192,256).
+// TMEM: per query tile q, columns q*256 + {S fp32 [0,128), P bf16x2 [128,192), O fp32 [192,256)}.
+constexpr uint32_t kTmemPerQ = 256;
+constexpr uint32_t kTmemCols = kTmemPerQ * kQPerCta;
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
-// Dynamic shared memory: Q tile, K and V stage rings (each 1024-byte aligned for the 128-byte
-// swizzle), then the barrier block. No static shared memory, so the dynamic base is the start
-// of the CTA's window (1024-aligned; checked at run time). Two CTAs fit in an SM's 228 KB.
-constexpr size_t kTilesBytes = (size_t)kTileBytes * (1 + 2 * kStages);
+// Dynamic shared memory: query tiles, K ring, V ring (each tile 1024-byte aligned for the
+// 128-byte swizzle), then the barrier block. No static shared memory, so the dynamic base is
+// the start of the CTA's window (1024-aligned; checked at run time).
+constexpr size_t kTilesBytes = (size_t)kTileBytes * (kQPerCta + kKStages + kVStages);
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: rescale O when the max grows > 2^8
 
 struct __align__(8) Shared {
-  uint64_t k_full[kStages];
-  uint64_t v_full[kStages];
-  uint64_t kv_empty[kStages];
-  uint64_t q_full;
-  uint64_t s_full;
-  uint64_t s_free;
-  uint64_t p_full;
-  uint64_t pv_done;
-  uint64_t lens[kStages];  // 8 valid-slot counts (bytes) per stage
+  uint64_t k_full[kKStages];
+  uint64_t k_empty[kKStages];
+  uint64_t v_full[kVStages];
+  uint64_t v_empty[kVStages];
+  // Valid-slot counts (one byte per page) of tile it live in lens[it % 4], published through
+  // lens_full[it % 4]; the producer cannot get 4 tiles ahead of the softmax warps because it
+  // waits for the V slot of tile it-3 (freed after P(it-3) V) before issuing tile it+1.
+  uint64_t lens_full[4];
+  uint64_t lens[4];
+  uint64_t q_full[kQPerCta];
+  uint64_t s_full[kQPerCta];
+  uint64_t s_free[kQPerCta];
+  uint64_t p_full[kQPerCta];
+  uint64_t pv_done[kQPerCta];
+  uint64_t turn[kQPerCta];  // exponential turns of the two softmax warpgroups
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -131,6 +164,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
       : "memory");
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
 #if GCA_SLEEP_WAIT
@@ -161,6 +205,27 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, Share
     if (mbar_try_wait(bar, parity)) return true;
     if (GCA_SLEEP_WAIT || (i & 63u) == 0u) {
       if (!drain && sh->abort_flag) return false;
+      if (global_timer() - t0 > kWaitNs) {
+        sh->abort_flag = 1;
+        atomicOr(err, GCA_DEVERR_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Spinning variant (no hardware suspend) for short, latency-critical hand-overs.
+__device__ __forceinline__ bool spin_phase(uint64_t* bar, uint32_t parity, Shared* sh,
+                                           uint32_t* err) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t i = 1;; ++i) {
+#if GCA_TURN_SPIN >= 2
+    __nanosleep(GCA_TURN_SPIN);  // back off: polls are shared-memory (MIO) instructions
+#endif
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((i & 255u) == 0u) {
+      if (sh->abort_flag) return false;
       if (global_timer() - t0 > kWaitNs) {
         sh->abort_flag = 1;
         atomicOr(err, GCA_DEVERR_WAIT_TIMEOUT);
@@ -263,19 +328,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
   const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
   asm volatile(
@@ -293,44 +345,29 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Packed fp32 pairs (sm_100 f32x2 instructions): one issue slot for two lanes of math.
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
 
-// 2^x on both bf16 halves (MUFU, two results per issue).
-__device__ __forceinline__ uint32_t ex2_bf2(uint32_t x) {
-  uint32_t y;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
-// acc_lo += low bf16 half of w, acc_hi += high half (mixed-precision adds, fp32 result).
-__device__ __forceinline__ void add_bf2(float& acc_lo, float& acc_hi, uint32_t w) {
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
-      : "+f"(acc_lo), "+f"(acc_hi)
-      : "r"(w));
+// 2^x on the FMA pipe. Range reduction x = j + r, j = round(x) (adding 1.5 * 2^23 leaves j in
+// the low mantissa bits), r in [-1/2, 1/2]; 2^r from a cubic fitted here for least maximum
+// relative error on [-1/2, 1/2] (Lawson-reweighted least squares); 2^j joins by an integer add
+// into the exponent field. Max relative error 7.5e-5 (float32), far below the bf16 rounding
+// of P that follows. x is clamped at -125 so the exponent add stays in range (masked -inf
+// scores give 2^-125 instead of 0).
+__device__ __forceinline__ float exp2_poly(float x) {
+  constexpr float kMagic = 12582912.0f;
+  constexpr float kC0 = 0.9999281167984009f, kC1 = 0.6932609677314758f;
+  constexpr float kC2 = 0.24261054396629333f, kC3 = 0.05517132207751274f;
+  x = fmaxf(x, -125.0f);
+  const float t = x + kMagic;
+  const float r = x - (t - kMagic);
+  float q = fmaf(kC3, r, kC2);
+  q = fmaf(q, r, kC1);
+  q = fmaf(q, r, kC0);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
@@ -381,13 +418,9 @@ __device__ __forceinline__ void resolve_page(const AttnParams& p, int lp, int fa
   }
 }
 
-struct Segment {
-  int unit, j0, j1;
-};
-
 // ------------------------------------------------------------------------- kernel
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -396,29 +429,36 @@ __global__ void __launch_bounds__(kThreads, 2)
     return;
   }
   Shared& sh = *reinterpret_cast<Shared*>(smem + kTilesBytes);
-  uint8_t* q_smem = smem;
-  uint8_t* k_smem = smem + kTileBytes;
-  uint8_t* v_smem = k_smem + kStages * kTileBytes;
+  uint8_t* q_smem = smem;                                   // kQPerCta query tiles
+  uint8_t* k_smem = smem + kQPerCta * kTileBytes;           // kKStages key tiles
+  uint8_t* v_smem = k_smem + kKStages * kTileBytes;         // kVStages value tiles
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&sh.k_full[s], 1);
-      mbar_init(&sh.v_full[s], 1);
-      mbar_init(&sh.kv_empty[s], 1);
+      mbar_init(&sh.k_empty[s], kQPerCta);
     }
-    mbar_init(&sh.q_full, kTileQ);
-    mbar_init(&sh.s_full, 1);
-    mbar_init(&sh.s_free, kTileQ);
-    mbar_init(&sh.p_full, kTileQ);
-    mbar_init(&sh.pv_done, 1);
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&sh.v_full[s], 1);
+      mbar_init(&sh.v_empty[s], kQPerCta);
+    }
+    for (int s = 0; s < 4; ++s) mbar_init(&sh.lens_full[s], 1);
+    for (int q = 0; q < kQPerCta; ++q) {
+      mbar_init(&sh.q_full[q], kTileQ);
+      mbar_init(&sh.s_full[q], 1);
+      mbar_init(&sh.s_free[q], kTileQ);
+      mbar_init(&sh.p_full[q], kTileQ);
+      mbar_init(&sh.pv_done[q], 1);
+      mbar_init(&sh.turn[q], kTileQ);
+    }
     sh.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
   }
-  if (warp == kWarpMma) {
+  if (warp == kWarpMma0) {
     asm volatile(
         "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
             smem_addr(&sh.tmem_base)),
@@ -438,20 +478,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     int fallback = 0;
     int flen = 0;
     resolve_page(p, 0, 0, &fallback, &flen);
-    uint32_t it = 0;
+    uint32_t it = 0, nk = 0, nv = 0;  // tiles walked; K and V copies issued
     bool ok = true;
     for (int64_t s = s_begin; s < s_end && ok;) {
-      const int u = (int)(s / p.n_tiles);
-      const int64_t seg_end = min(s_end, (int64_t)(u + 1) * p.n_tiles);
-      const int h = u / p.n_qt;
-      for (int j = (int)(s - (int64_t)u * p.n_tiles); j < (int)(seg_end - (int64_t)u * p.n_tiles);
+      const int u2 = (int)(s / p.n_tiles);
+      const int64_t seg_end = min(s_end, (int64_t)(u2 + 1) * p.n_tiles);
+      const int h = u2 / p.n_pairs;
+      for (int j = (int)(s - (int64_t)u2 * p.n_tiles); j < (int)(seg_end - (int64_t)u2 * p.n_tiles);
            ++j, ++it) {
-        const int stage = it % kStages;
-        const uint32_t use = it / kStages;
-        if (use > 0 && !warp_wait(&sh.kv_empty[stage], (use - 1) & 1u, &sh, p.err)) {
-          ok = false;
-          break;
-        }
+        const int ks = it % kKStages, vs = it % kVStages;
+        const uint32_t kuse = it / kKStages, vuse = it / kVStages;
         int page = 0, len = 0;
         if (lane < kPagesPerTile) resolve_page(p, j * kPagesPerTile + lane, fallback, &page, &len);
         if (page < 0 || page >= p.num_pages) {
@@ -464,78 +500,101 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int k = 0; k < kPagesPerTile; ++k) {
           lens |= (uint64_t)(uint32_t)__shfl_sync(0xffffffffu, len, k) << (8 * k);
         }
+        const int row = (page * p.H + h) * kPageSize;
+        if (kuse > 0 && !warp_wait(&sh.k_empty[ks], (kuse - 1) & 1u, &sh, p.err)) {
+          ok = false;
+          break;
+        }
         if (lane == 0) {
-          sh.lens[stage] = lens;
-          mbar_arrive_expect_tx(&sh.k_full[stage], kTileBytes);
-          mbar_arrive_expect_tx(&sh.v_full[stage], kTileBytes);
+          TRACE(0, it);
+          sh.lens[it & 3] = lens;
+          mbar_arrive(&sh.lens_full[it & 3]);
+          mbar_arrive_expect_tx(&sh.k_full[ks], kTileBytes);
         }
         __syncwarp();
         if (lane < kPagesPerTile) {
-          const int row = (page * p.H + h) * kPageSize;
-          tma_load_2d(smem_addr(k_smem + stage * kTileBytes + lane * kPageBytes), &tm_k, 0, row,
-                      &sh.k_full[stage]);
-          tma_load_2d(smem_addr(v_smem + stage * kTileBytes + lane * kPageBytes), &tm_v, 0, row,
-                      &sh.v_full[stage]);
+          tma_load_2d(smem_addr(k_smem + ks * kTileBytes + lane * kPageBytes), &tm_k, 0, row,
+                      &sh.k_full[ks]);
         }
+        ++nk;
+        if (vuse > 0 && !warp_wait(&sh.v_empty[vs], (vuse - 1) & 1u, &sh, p.err)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          TRACE(1, it);
+          mbar_arrive_expect_tx(&sh.v_full[vs], kTileBytes);
+        }
+        __syncwarp();
+        if (lane < kPagesPerTile) {
+          tma_load_2d(smem_addr(v_smem + vs * kTileBytes + lane * kPageBytes), &tm_v, 0, row,
+                      &sh.v_full[vs]);
+        }
+        ++nv;
       }
       s = seg_end;
     }
-    // Drain: wait until the last issued copies have landed before the CTA can exit.
-    const uint32_t issued = it;
-    const uint32_t first = issued > (uint32_t)kStages ? issued - kStages : 0u;
-    for (uint32_t q = first; q < issued; ++q) {
-      const int stage = q % kStages;
-      const uint32_t use = q / kStages;
-      warp_wait(&sh.k_full[stage], use & 1u, &sh, p.err, true);
-      warp_wait(&sh.v_full[stage], use & 1u, &sh, p.err, true);
+    // Drain: wait until the copies issued last have landed before the CTA can exit.
+    for (uint32_t q = nk > (uint32_t)kKStages ? nk - kKStages : 0u; q < nk; ++q) {
+      warp_wait(&sh.k_full[q % kKStages], (q / kKStages) & 1u, &sh, p.err, true);
     }
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issuer
-    // Per tile j: S(j) = Q K_j^T is issued as soon as the softmax warps have read S(j-1) out of
-    // TMEM, so it runs while they compute P(j-1); then O += P(j-1) V_(j-1).
+    for (uint32_t q = nv > (uint32_t)kVStages ? nv - kVStages : 0u; q < nv; ++q) {
+      warp_wait(&sh.v_full[q % kVStages], (q / kVStages) & 1u, &sh, p.err, true);
+    }
+  } else if (warp == kWarpMma0 || warp == kWarpMma0 + 1) {
+    // ------------------------------------------------------------ MMA issuers, one per query
+    // tile (a thread issues about one tcgen05.mma per 60 cycles, so one thread could not keep
+    // the tensor core fed for both tiles). Per key tile j: S(j) = Q K_j^T as soon as the
+    // softmax warps have read S(j-1); then O += P(j-1) V_(j-1).
+    const int qq = warp - kWarpMma0;
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16(kTileK, false);
       constexpr uint32_t kIdescPV = idesc_bf16(kHeadDim, true);
-      const uint64_t q_desc = sw128_desc(smem_addr(q_smem), 16, 1024);
+      const uint32_t tq = tmem + kTmemPerQ * qq;
+      const uint64_t q_desc = sw128_desc(smem_addr(q_smem + qq * kTileBytes), 16, 1024);
       uint32_t it = 0, seg = 0;
       bool ok = true;
       for (int64_t s = s_begin; s < s_end && ok; ++seg) {
-        const int u = (int)(s / p.n_tiles);
-        const int64_t seg_end = min(s_end, (int64_t)(u + 1) * p.n_tiles);
-        const int j0 = (int)(s - (int64_t)u * p.n_tiles);
-        const int j1 = (int)(seg_end - (int64_t)u * p.n_tiles);
-        if (!wait_phase(&sh.q_full, seg & 1u, &sh, p.err)) break;
+        const int u2 = (int)(s / p.n_tiles);
+        const int64_t seg_end = min(s_end, (int64_t)(u2 + 1) * p.n_tiles);
+        const int j0 = (int)(s - (int64_t)u2 * p.n_tiles);
+        const int j1 = (int)(seg_end - (int64_t)u2 * p.n_tiles);
+        if (!wait_phase(&sh.q_full[qq], seg & 1u, &sh, p.err)) break;
         tc_fence_after();
         for (int j = j0; j <= j1; ++j) {
           if (j < j1) {
-            const int stage = it % kStages;
-            const uint32_t use = it / kStages;
-            if (!wait_phase(&sh.k_full[stage], use & 1u, &sh, p.err)) { ok = false; break; }
-            if (j > j0 && !wait_phase(&sh.s_free, (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
+            const int ks = it % kKStages;
+            if (!wait_phase(&sh.k_full[ks], (it / kKStages) & 1u, &sh, p.err)) { ok = false; break; }
+            if (j > j0 && !wait_phase(&sh.s_free[qq], (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t k_desc = sw128_desc(smem_addr(k_smem + stage * kTileBytes), 16, 1024);
+            if (qq == 0) TRACE(2, it);
+            const uint64_t k_desc = sw128_desc(smem_addr(k_smem + ks * kTileBytes), 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < kHeadDim / 16; ++kk) {
               // +32 bytes along K inside the swizzled 128-byte rows
-              mma_ss(tmem + kColS, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
+              mma_ss(tq + kColS, q_desc + 2 * kk, k_desc + 2 * kk, kIdescS, kk > 0 ? 1u : 0u);
             }
-            mma_commit(&sh.s_full);
+            mma_commit(&sh.s_full[qq]);
+            mma_commit(&sh.k_empty[ks]);
+            if (qq == 0) TRACE(3, it);
           }
           if (j > j0) {
             const uint32_t pit = it - 1;  // tile j-1
-            const int pst = pit % kStages;
-            if (!wait_phase(&sh.p_full, pit & 1u, &sh, p.err)) { ok = false; break; }
-            if (!wait_phase(&sh.v_full[pst], (pit / kStages) & 1u, &sh, p.err)) { ok = false; break; }
+            const int vs = pit % kVStages;
+            if (!wait_phase(&sh.p_full[qq], pit & 1u, &sh, p.err)) { ok = false; break; }
+            if (!wait_phase(&sh.v_full[vs], (pit / kVStages) & 1u, &sh, p.err)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t v_desc = sw128_desc(smem_addr(v_smem + pst * kTileBytes), 16384, 1024);
+            if (qq == 0) TRACE(4, pit);
+            const uint64_t v_desc = sw128_desc(smem_addr(v_smem + vs * kTileBytes), 16384, 1024);
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk) {
               // 16 keys: 2048 bytes of V, 8 TMEM columns of packed P
-              mma_ts(tmem + kColO, tmem + kColP + 8 * kk, v_desc + 128 * kk, kIdescPV,
+              mma_ts(tq + kColO, tq + kColP + 8 * kk, v_desc + 128 * kk, kIdescPV,
                      (j - 1 > j0 || kk > 0) ? 1u : 0u);
             }
-            mma_commit(&sh.pv_done);
-            mma_commit(&sh.kv_empty[pst]);
+            mma_commit(&sh.pv_done[qq]);
+            mma_commit(&sh.v_empty[vs]);
+            if (qq == 0) TRACE(5, pit);
           }
           if (j < j1) ++it;
         }
@@ -544,46 +603,55 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax warps 0-3
-    const int r = threadIdx.x;  // query row within the tile == TMEM lane
-    const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
-    uint32_t it = 0;
+    // ------------------------------------------------------------ softmax warpgroups
+    // Warpgroup qq (warps 4*qq .. 4*qq+3) owns query tile qq; thread r owns row r (TMEM lane r).
+    // The two warpgroups take turns for the exponentials (MUFU-bound) so that one computes
+    // them while the other waits for S, loads it and reduces the row max.
+    const int qq = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t t_row = tmem + kTmemPerQ * qq + ((uint32_t)((warp & 3) * 32) << 16);
+    uint8_t* q_tile = q_smem + qq * kTileBytes;
+    uint32_t it = 0, turns = 0;
     bool ok = true;
+#if GCA_TURNS
+    if (qq == 1) mbar_arrive(&sh.turn[0]);  // the first turn goes to query tile 0
+#endif
     for (int64_t s = s_begin; s < s_end && ok;) {
-      const int u = (int)(s / p.n_tiles);
-      const int64_t seg_end = min(s_end, (int64_t)(u + 1) * p.n_tiles);
-      const int j0 = (int)(s - (int64_t)u * p.n_tiles);
-      const int j1 = (int)(seg_end - (int64_t)u * p.n_tiles);
-      const int h = u / p.n_qt;
-      const int qt = u % p.n_qt;
+      const int u2 = (int)(s / p.n_tiles);
+      const int64_t seg_end = min(s_end, (int64_t)(u2 + 1) * p.n_tiles);
+      const int j0 = (int)(s - (int64_t)u2 * p.n_tiles);
+      const int j1 = (int)(seg_end - (int64_t)u2 * p.n_tiles);
+      const int h = u2 / p.n_pairs;
+      const int qt = (u2 % p.n_pairs) * kQPerCta + qq;
       const int qi = qt * kTileQ + r;
 
       // Q row -> shared memory, 128-byte swizzle (16-byte chunk c of row r at c ^ (r % 8))
       {
+        const bool valid = qt < p.n_qt && qi < p.T;
         const uint4* src = p.q + ((int64_t)qi * p.H + h) * 8;
-        uint8_t* row = q_smem + r * 128;
+        uint8_t* row = q_tile + r * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          uint4 v = qi < p.T ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+          uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
           *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = v;
         }
         fence_proxy_async_smem();
-        mbar_arrive(&sh.q_full);
+        mbar_arrive(&sh.q_full[qq]);
       }
 
       float m_run = -INFINITY;  // running row max, log2 units (scaled)
       float l_run = 0.f;        // running row sum relative to m_run
       for (int j = j0; j < j1; ++j, ++it) {
-        if (!warp_wait(&sh.s_full, it & 1u, &sh, p.err)) { ok = false; break; }
+        if (!warp_wait(&sh.s_full[qq], it & 1u, &sh, p.err)) { ok = false; break; }
+        if (!warp_wait(&sh.lens_full[it & 3], (it >> 2) & 1u, &sh, p.err)) { ok = false; break; }
+        const uint64_t lens = sh.lens[it & 3];
+        if (r == 0 && qq == 0) TRACE(6, it);
         tc_fence_after();
         float sv[kTileK];
         tmem_ld128(t_row + kColS, sv);
         tc_fence_before();
-        mbar_arrive(&sh.s_free);  // the MMA warp may now compute the next S
+        mbar_arrive(&sh.s_free[qq]);  // the MMA warp may now compute the next S
 
-        const int stage = it % kStages;
-        if (!warp_wait(&sh.k_full[stage], (it / kStages) & 1u, &sh, p.err)) { ok = false; break; }
-        const uint64_t lens = sh.lens[stage];
         if (lens != 0x1010101010101010ull) {
 #pragma unroll
           for (int pg = 0; pg < kPagesPerTile; ++pg) {
@@ -617,119 +685,100 @@ __global__ void __launch_bounds__(kThreads, 2)
           m_new = tile_max;
           alpha = ex2(m_run - m_new);
         }
-        // P = 2^(s*c - m), rounded to bf16 pairs for P V; the row sum accumulates the fp32
-        // values (the bf16 path sums the rounded values instead).
-        const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t nm2 = f2_pack(-m_new, -m_new);
+        if (j > j0) {
+          // P V of the previous tile must be done before P is overwritten or O rescaled
+          if (!warp_wait(&sh.pv_done[qq], (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
+          tc_fence_after();
+        }
+        // P = 2^(s*c - m), inside this warpgroup's turn on MUFU: scale-subtract, exponentials,
+        // bf16 packing, row sum and TMEM stores, 32 columns at a time. The turn passes to the
+        // other warpgroup GCA_TURN_EARLY chunks before the end so that its first exponentials
+        // queue behind this group's last ones.
+#if GCA_TURNS && GCA_TURN_SPIN
+        if (!__all_sync(0xffffffffu, spin_phase(&sh.turn[qq], turns & 1u, &sh, p.err))) {
+          ok = false;
+          break;
+        }
+#elif GCA_TURNS
+        if (!warp_wait(&sh.turn[qq], turns & 1u, &sh, p.err)) { ok = false; break; }
+#endif
+        if (r == 0 && qq == 0) TRACE(7, it);
         const float neg_m = -m_new;
-        uint32_t pk[kTileK / 2];
+#pragma unroll
+        for (int e = 0; e < kTileK; ++e) sv[e] = fmaf(sv[e], p.scale_log2, neg_m);
         float rs[8];
 #pragma unroll
         for (int a = 0; a < 8; ++a) rs[a] = 0.f;
-#if GCA_STAGED
 #pragma unroll
-        for (int e = 0; e < kTileK; ++e) sv[e] = fmaf(sv[e], p.scale_log2, neg_m);
-#if GCA_EXP_BF16
+        for (int chunk = 0; chunk < kTileK / 32; ++chunk) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < kTileK / 2; ++c) pk[c] = ex2_bf2(pack_bf2(sv[2 * c], sv[2 * c + 1]));
-#pragma unroll
-        for (int c = 0; c < kTileK / 2; ++c) add_bf2(rs[2 * (c & 3)], rs[2 * (c & 3) + 1], pk[c]);
-#else
-#pragma unroll
-        for (int e = 0; e < kTileK; ++e) sv[e] = ex2(sv[e]);
-#pragma unroll
-        for (int c = 0; c < kTileK / 2; ++c) {
-          pk[c] = pack_bf2(sv[2 * c], sv[2 * c + 1]);
-          rs[2 * (c & 3)] += sv[2 * c];
-          rs[2 * (c & 3) + 1] += sv[2 * c + 1];
+          for (int c = 0; c < 16; ++c) {
+            const int e = 32 * chunk + 2 * c;
+            const bool poly = c < GCA_POLY_PAIRS;
+            const float e0 = poly ? exp2_poly(sv[e]) : ex2(sv[e]);
+            const float e1 = poly ? exp2_poly(sv[e + 1]) : ex2(sv[e + 1]);
+            pk[c] = pack_bf2(e0, e1);
+            rs[2 * (c & 3)] += e0;
+            rs[2 * (c & 3) + 1] += e1;
+          }
+          tmem_st16(t_row + kColP + 16 * chunk, reinterpret_cast<const float*>(pk));
+          if (GCA_TURNS && chunk == kTileK / 32 - 1 - GCA_TURN_EARLY) mbar_arrive(&sh.turn[qq ^ 1]);
         }
-#endif
-#else
+        ++turns;
+        if (r == 0 && qq == 0) TRACE(8, it);
+        // Lazy rescale of O (rare): after the scores are dead, before P V(j) is issued.
+        if (j > j0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-        for (int c = 0; c < kTileK / 2; ++c) {
-          float x0, x1;
-#if GCA_FMA2
-          f2_unpack(f2_fma(f2_pack(sv[2 * c], sv[2 * c + 1]), c2, nm2), x0, x1);
-#else
-          x0 = fmaf(sv[2 * c], p.scale_log2, neg_m);
-          x1 = fmaf(sv[2 * c + 1], p.scale_log2, neg_m);
-#endif
-#if GCA_EXP_BF16
-          pk[c] = ex2_bf2(pack_bf2(x0, x1));
-#if GCA_SUM_MIXED
-          add_bf2(rs[2 * (c & 3)], rs[2 * (c & 3) + 1], pk[c]);
-#else
-          rs[2 * (c & 3)] += __uint_as_float(pk[c] << 16);
-          rs[2 * (c & 3) + 1] += __uint_as_float(pk[c] & 0xffff0000u);
-#endif
-#else
-          const float e0 = ex2(x0), e1 = ex2(x1);
-          pk[c] = pack_bf2(e0, e1);
-          rs[2 * (c & 3)] += e0;
-          rs[2 * (c & 3) + 1] += e1;
-#endif
-        }
-#endif
-        (void)c2;
-        (void)nm2;
-        (void)neg_m;
-        const float row_sum =
-            ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
-
-        if (j > j0) {
-          // P V of the previous tile must be done before P is overwritten or O rescaled
-          if (!warp_wait(&sh.pv_done, (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+          for (int c = 0; c < kHeadDim / 16; ++c) {
+            float o[16];
+            tmem_ld16(t_row + kColO + 16 * c, o);
 #pragma unroll
-            for (int c = 0; c < kHeadDim / 16; ++c) {
-              float o[16];
-              tmem_ld16(t_row + kColO + 16 * c, o);
-#pragma unroll
-              for (int a = 0; a < 16; ++a) o[a] *= alpha;
-              tmem_st16(t_row + kColO + 16 * c, o);
-            }
-            tmem_wait_st();
+            for (int a = 0; a < 16; ++a) o[a] *= alpha;
+            tmem_st16(t_row + kColO + 16 * c, o);
           }
         }
+        const float row_sum =
+            ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
         l_run = l_run * alpha + row_sum;
         m_run = m_new;
-        tmem_st32(t_row + kColP, pk);
-        tmem_st32(t_row + kColP + 32, pk + 32);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&sh.p_full);
+        mbar_arrive(&sh.p_full[qq]);
+        if (r == 0 && qq == 0) TRACE(9, it);
       }
       if (!ok) break;
 
       // ---- epilogue
-      if (!warp_wait(&sh.pv_done, (it - 1) & 1u, &sh, p.err)) break;
+      if (!warp_wait(&sh.pv_done[qq], (it - 1) & 1u, &sh, p.err)) break;
       tc_fence_after();
       float o[kHeadDim];
       tmem_ld64(t_row + kColO, o);
       tc_fence_before();
-      if (j0 == 0 && j1 == p.n_tiles) {
-        if (qi < p.T) {
-          const float inv = 1.f / l_run;
-          uint4* dst = p.out + ((int64_t)qi * p.H + h) * 8;
+      if (qt < p.n_qt) {
+        if (j0 == 0 && j1 == p.n_tiles) {
+          if (qi < p.T) {
+            const float inv = 1.f / l_run;
+            uint4* dst = p.out + ((int64_t)qi * p.H + h) * 8;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4 w;
-            w.x = pack_bf2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
-            w.y = pack_bf2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
-            w.z = pack_bf2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
-            w.w = pack_bf2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
-            dst[c] = w;
+            for (int c = 0; c < 8; ++c) {
+              uint4 w;
+              w.x = pack_bf2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
+              w.y = pack_bf2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
+              w.z = pack_bf2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
+              w.w = pack_bf2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
+              dst[c] = w;
+            }
           }
-        }
-      } else {
-        const int64_t slot = (int64_t)blockIdx.x + u;
-        float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * kTileQ + r) * kHeadDim);
+        } else {
+          const int64_t slot = part_slot(blockIdx.x, u2, qq);
+          float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * kTileQ + r) * kHeadDim);
 #pragma unroll
-        for (int c = 0; c < kHeadDim / 4; ++c) {
-          dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          for (int c = 0; c < kHeadDim / 4; ++c) {
+            dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          }
+          p.part_ml[slot * kTileQ + r] = make_float2(m_run, l_run);
         }
-        p.part_ml[slot * kTileQ + r] = make_float2(m_run, l_run);
       }
       s = seg_end;
     }
@@ -737,39 +786,43 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpMma) {
+  if (warp == kWarpMma0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols));
   }
 }
 
-// Merges the partial records of every split unit: weights 2^(m_s - M), M = max_s m_s.
-// Two threads per query row, 32 output columns each.
+// Merges the partial records of every split (head, query tile): weights 2^(m_s - M),
+// M = max_s m_s. Two threads per query row, 32 output columns each.
 constexpr int kCombineThreads = 2 * kTileQ;
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const AttnParams p) {
-  const int u = blockIdx.x;
+  const int u = blockIdx.x;  // (head, query tile)
   const int r = threadIdx.x >> 1;
   const int half = threadIdx.x & 1;
-  const int64_t first = (int64_t)u * p.n_tiles;
+  const int h = u / p.n_qt;
+  const int qt = u % p.n_qt;
+  const int u2 = h * p.n_pairs + qt / kQPerCta;
+  const int qq = qt % kQPerCta;
+  const int64_t first = (int64_t)u2 * p.n_tiles;
   const int64_t c0 = cta_of_step(first, p.total, p.grid);
   const int64_t c1 = cta_of_step(first + p.n_tiles - 1, p.total, p.grid);
   if (c0 == c1) return;
-  const int h = u / p.n_qt;
-  const int qi = (u % p.n_qt) * kTileQ + r;
+  const int qi = qt * kTileQ + r;
   if (qi >= p.T) return;
   float M = -INFINITY;
-  for (int64_t c = c0; c <= c1; ++c) M = fmaxf(M, p.part_ml[(c + u) * kTileQ + r].x);
+  for (int64_t c = c0; c <= c1; ++c) M = fmaxf(M, p.part_ml[part_slot(c, u2, qq) * kTileQ + r].x);
   float acc[32];
 #pragma unroll
   for (int a = 0; a < 32; ++a) acc[a] = 0.f;
   float L = 0.f;
   for (int64_t c = c0; c <= c1; ++c) {
-    const float2 ml = p.part_ml[(c + u) * kTileQ + r];
+    const int64_t slot = part_slot(c, u2, qq);
+    const float2 ml = p.part_ml[slot * kTileQ + r];
     const float w = ex2(ml.x - M);
     L += w * ml.y;
-    const float4* src = reinterpret_cast<const float4*>(
-        p.part_o + ((c + u) * kTileQ + r) * kHeadDim + 32 * half);
+    const float4* src =
+        reinterpret_cast<const float4*>(p.part_o + (slot * kTileQ + r) * kHeadDim + 32 * half);
 #pragma unroll
     for (int a = 0; a < 8; ++a) {
       const float4 v = __ldcg(src + a);
@@ -798,17 +851,8 @@ cudaError_t attn_prepare(int* ctas_per_sm) {
   cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           (int)cudaSharedmemCarveoutMaxShared);
-  if (e != cudaSuccess) return e;
-  int n = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel, kThreads, kSmemBytes);
-  if (e != cudaSuccess) return e;
-  // Registers and shared memory admit two CTAs per SM and the two share the SM's 512 TMEM
-  // columns (256 each); the occupancy query ignores the shared-memory carveout, so it is only
-  // a lower bound here.
-  (void)n;
-  *ctas_per_sm = 2;
+  // One CTA per SM: it holds all 512 TMEM columns (two query tiles).
+  *ctas_per_sm = 1;
   return cudaSuccess;
 }
 
@@ -824,3 +868,10 @@ cudaError_t launch_combine(const AttnParams& p, cudaStream_t s) {
 }
 
 }  // namespace gca
+
+#if GCA_TRACE
+extern "C" int gca_debug_trace(void* host, size_t bytes) {
+  if (bytes > sizeof(gca::g_trace)) bytes = sizeof(gca::g_trace);
+  return (int)cudaMemcpyFromSymbol(host, gca::g_trace, bytes);
+}
+#endif

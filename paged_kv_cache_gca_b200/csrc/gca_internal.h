@@ -9,6 +9,8 @@
 
 #include "../../include/gca.h"
 
+struct gca_cache;
+
 namespace gca {
 
 constexpr int kHeadDim = 64;
@@ -31,7 +33,8 @@ struct Layout {
   size_t traj_pages;         // int32 [traj_cap_pages]
   size_t slot_map;           // int32 [T]
   size_t kept;               // int32 [kMaxKeep]
-  size_t rope_t, rope_y, rope_x;  // float2 (cos, sin) tables
+  size_t rope_t;             // float2 (cos, sin) [max_frames][nt]: time band per frame
+  size_t rope_tok;           // float2 (cos, sin) [T][ny + nx]: spatial bands per token
   size_t err;                // uint32 sticky device error word
   size_t part_o;             // float [part_slots][128][64]
   size_t part_ml;            // float2 [part_slots][128]
@@ -55,11 +58,10 @@ struct InitParams {
   const int32_t* user_free;  // may be null
   int32_t* kept;
   float2* rope_t;
-  float2* rope_y;
-  float2* rope_x;
+  float2* rope_tok;
   uint32_t* err;
   int32_t num_pages;
-  int32_t max_frames, grid_h, grid_w;
+  int32_t max_frames, grid_h, grid_w, num_special, T;
   int32_t nt, ny, nx;
   int32_t keep;
   double base;
@@ -79,22 +81,23 @@ struct AppendParams {
   int32_t* slot_map;
   const int32_t* kept;
   const float2* rope_t;
-  const float2* rope_y;
-  const float2* rope_x;
+  const float2* rope_tok;
   uint32_t* err;
   int64_t t;
-  int64_t free_head;
-  int64_t free_tail;
   int64_t traj_len;
-  int32_t T, H, S, grid_w, ppf, num_pages;
-  int32_t nt, ny, nx;
+  int32_t head_pos;           // free_head mod num_pages: ring position of the first pop
+  int32_t tail_pos;           // free_tail mod num_pages: ring position of the first push
+  int32_t T, H, ppf, num_pages;
+  int32_t nt, nyx;            // RoPE pairs of the time band; of the two spatial bands
   int32_t evict_frame;        // -1: nothing leaves the window
   int32_t K;                  // kept tokens copied (0 if no eviction)
   int32_t traj_pages_before;  // trajectory pages before this step
   int32_t n_pop_traj;         // trajectory pages popped by this step
   int32_t zero_slots;         // slots zero-filled at the end of the last new trajectory page
-  // item ranges of the single launch
-  int64_t n_tok_items, n_evict_items, n_zero_items, n_push_items, n_traj_items, n_items;
+  // launch shape: token blocks of (8 chunks, H heads, tok_per_block tokens) threads, then
+  // blocks of kAuxThreads for the eviction items
+  int32_t tok_per_block, n_tok_blocks;
+  int64_t n_evict_items, n_zero_items, n_push_items, n_traj_items, n_aux_items;
 };
 
 struct AttnParams {
@@ -114,8 +117,10 @@ struct AttnParams {
   int32_t n_lp;          // logical pages walked
   int32_t n_tiles;       // 128-key tiles
   int32_t n_qt;          // 128-query tiles per head
-  int32_t units;         // H * n_qt
-  int64_t total;         // units * n_tiles
+  int32_t units;         // H * n_qt: (head, query tile) pairs, the combine grid
+  int32_t n_pairs;       // query-tile pairs per head (a CTA works on two tiles of one head)
+  int32_t units2;        // H * n_pairs: work units of the attention kernel
+  int64_t total;         // units2 * n_tiles
   int32_t grid;
   float scale_log2;      // log2(e) / sqrt(D)
 };
@@ -132,11 +137,21 @@ cudaError_t launch_attn(const CUtensorMap& tk, const CUtensorMap& tv, const Attn
 cudaError_t launch_combine(const AttnParams& p, cudaStream_t s);
 
 // Split bookkeeping shared by the attention and combine kernels: CTA c owns the flattened
-// (unit, tile) steps [c*total/grid, (c+1)*total/grid); the CTA that holds step s is
-// ceil((s+1)*grid/total) - 1, and (unit u, CTA c) writes its partial result to slot c + u.
+// (pair unit, key tile) steps [c*total/grid, (c+1)*total/grid); the CTA that holds step s is
+// ceil((s+1)*grid/total) - 1, and (CTA c, pair unit u2, query tile q of the pair) writes its
+// partial result to slot 2*(c + u2) + q. Over a launch the slots stay below 2*(grid + units2).
 __host__ __device__ inline int64_t cta_of_step(int64_t s, int64_t total, int64_t grid) {
   return ((s + 1) * grid + total - 1) / total - 1;
 }
+__host__ __device__ inline int64_t part_slot(int64_t cta, int64_t u2, int q) {
+  return 2 * (cta + u2) + q;
+}
+
+// Fills the frame-dependent fields of p for gca_attend of frame t (visible page ranges, tiles,
+// work split) with at most max_slots partial-record slots; returns false if even one CTA per
+// work unit does not fit. *split: some unit spans several CTAs, so the combine kernel must run.
+bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams* p,
+                    bool* split, int64_t* visible_keys);
 
 }  // namespace gca
 

@@ -29,7 +29,6 @@ constexpr size_t kNoallocScratchBytes = (size_t)16 << 20;
 constexpr size_t kSlotOBytes = (size_t)kTileQ * kHeadDim * sizeof(float);
 constexpr size_t kSlotMLBytes = (size_t)kTileQ * sizeof(float2);
 constexpr int kNoallocSlots = (int)(kNoallocScratchBytes / (kSlotOBytes + kSlotMLBytes));
-constexpr int kMinStepsPerCtaNoalloc = 16;
 constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_attend_scratch[kNoallocScratchBytes];
@@ -63,65 +62,18 @@ extern "C" gca_status gca_attend_noalloc(gca_cache* c, int64_t t, const void* q_
   if (c->frames == 0 || t != c->frames - 1) return GCA_ERR_FRAME_ORDER;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != c->device) return GCA_ERR_INVALID_ARG;
-  const Layout& L = c->lay;
-  const gca_config& cf = c->cfg;
-  const int units = cf.num_heads * L.n_qt;
-  // The partial records of one call take (grid + units) slots; at least one CTA must fit.
-  if (units + 1 > kNoallocSlots) return GCA_ERR_UNSUPPORTED;
+  // The partial records of one call must fit the array (at least one CTA per work unit).
+  AttnParams p;
+  bool split = false;
+  int64_t nk = 0;
+  if (!plan_attention(c, t, kNoallocSlots, &p, &split, &nk)) return GCA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   if (scratch_address(dev, &scratch) != cudaSuccess) return GCA_ERR_CUDA;
-
-  int64_t na_frames, w0, nwf;
-  if (t < cf.anchor_frames) {
-    na_frames = t + 1;
-    w0 = 0;
-    nwf = 0;
-  } else {
-    na_frames = cf.anchor_frames;
-    w0 = std::max<int64_t>(cf.anchor_frames, t - cf.window_frames + 1);
-    nwf = t - w0 + 1;
-  }
-  AttnParams p;
-  std::memset(&p, 0, sizeof(p));
   p.q = static_cast<const uint4*>(q_rot);
   p.out = static_cast<uint4*>(out);
   p.part_o = static_cast<float*>(scratch);
   p.part_ml = reinterpret_cast<float2*>(static_cast<char*>(scratch) +
                                         (size_t)kNoallocSlots * kSlotOBytes);
-  p.frame_pages = reinterpret_cast<const int32_t*>(c->ws + L.frame_pages);
-  p.traj_pages = reinterpret_cast<const int32_t*>(c->ws + L.traj_pages);
-  p.err = reinterpret_cast<uint32_t*>(c->ws + L.err);
-  p.T = L.T;
-  p.H = cf.num_heads;
-  p.ppf = L.ppf;
-  p.last_len = L.last_len;
-  p.num_pages = cf.num_pages;
-  p.na_pages = (int32_t)(na_frames * L.ppf);
-  p.win_base = (int32_t)(w0 * L.ppf);
-  p.nw_pages = (int32_t)(nwf * L.ppf);
-  p.n_traj_pages = c->traj_pages;
-  p.traj_tail_len =
-      c->traj_pages > 0 ? (int32_t)(c->traj_len - (int64_t)(c->traj_pages - 1) * kPageSize) : 0;
-  p.n_lp = p.na_pages + p.nw_pages + p.n_traj_pages;
-  p.n_tiles = (p.n_lp + kPagesPerTile - 1) / kPagesPerTile;
-  p.n_qt = L.n_qt;
-  p.units = units;
-  p.total = (int64_t)p.units * p.n_tiles;
-  int64_t gmax = std::min<int64_t>(kMaxGrid, (int64_t)c->sms * c->ctas_per_sm);
-  gmax = std::min<int64_t>(gmax, kNoallocSlots - units);  // partial slots must fit the array
-  int64_t g = (p.total + kMinStepsPerCtaNoalloc - 1) / kMinStepsPerCtaNoalloc;
-  g = std::max<int64_t>(g, std::min<int64_t>(p.units, gmax));
-  g = std::min<int64_t>(g, gmax);
-  g = std::min<int64_t>(g, p.total);
-  p.grid = (int32_t)g;
-  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)cf.head_dim));
-
-  bool split = false;
-  for (int u = 0; u < p.units && !split; ++u) {
-    const int64_t first = (int64_t)u * p.n_tiles;
-    split = cta_of_step(first, p.total, p.grid) !=
-            cta_of_step(first + p.n_tiles - 1, p.total, p.grid);
-  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (launch_attn(c->tm_k, c->tm_v, p, s) != cudaSuccess) return GCA_ERR_CUDA;
   if (split && launch_combine(p, s) != cudaSuccess) return GCA_ERR_CUDA;

@@ -52,7 +52,7 @@ def test_noalloc_matches_attend_on_two_calls_in_a_row():
 
 
 def test_noalloc_rejects_frames_beyond_its_scratch():
-    # 64 heads x 8 query tiles need 512 partial-record slots at least: more than the array holds
+    # 64 heads x 4 pairs of query tiles need 2 x 256 partial records at least: the array holds 496
     w = gi.workload("w16_320").replace(num_heads=64, num_pages=64, frames=1, max_frames=4)
     cache = gca.GcaCache(gca.config_for(w))
     shape = (w.tokens_per_frame, w.num_heads, w.head_dim)
