@@ -230,6 +230,7 @@ def run_ours(args, rank, world, device):
 
     # ---- end-to-end through the public API with host buffers (pinned), copies timed
     e2e = run_e2e(args, w, cache, ring_host, device, stream, world)
+    batched = run_batched_append(ring, device, stream) if world == 1 else None
 
     res = {
         "elapsed_ms": elapsed_ms,
@@ -241,9 +242,71 @@ def run_ours(args, rank, world, device):
         "clocks": clk.summary(),
         "e2e": e2e,
         "frames": nframes,
+        "batched_append": batched,
     }
     cache.close()
     return w, res
+
+
+def run_batched_append(ring, device, stream, warm=16, timed=32):
+    """Append bandwidth of one launch over all caches of the 24-layer x 4-stream stack
+    (gca_append_frames): 96 caches, 12.34 MB each per frame, 1.18 GB per launch. Inputs come
+    from the device ring (frame of cache c at step t: slot (96 t + c) mod R, so one launch reads
+    590 MB); every cache writes its own q_rot buffer. The argument arrays of every launch are
+    built before the timed region, and the stream is kept busy (a device-side sleep) while the
+    host enqueues the timed launches, so the events time the launches back to back."""
+    import ctypes
+
+    import paged_kv_cache_gca_b200 as gca
+
+    w = gi.workload("stack24x4")
+    n = w.num_layers * w.num_streams
+    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    R = ring.shape[0]
+    fb = T * H * D * 2
+    with torch.cuda.stream(stream):
+        caches = [gca.GcaCache(gca.config_for(w, gi.rope_base_for_layer(w, c % w.num_layers)),
+                               stream=stream) for c in range(n)]
+    q_rot = [torch.empty((T, H, D), dtype=torch.bfloat16, device=device) for _ in range(n)]
+    VP, I64 = ctypes.c_void_p, ctypes.c_int64
+    handles = (VP * n)(*[c.handle for c in caches])
+    qr = (VP * n)(*[x.data_ptr() for x in q_rot])
+    base = ring.data_ptr()  # [R, 3, T, H, D] contiguous
+
+    def call_args(t):
+        slots = [(n * t + c) % R for c in range(n)]
+        ptrs = [(VP * n)(*[base + (3 * s + j) * fb for s in slots]) for j in range(3)]
+        return (handles, n, (I64 * n)(*([t] * n)), ptrs[0], ptrs[1], ptrs[2], qr,
+                stream.cuda_stream)
+
+    L = gca.lib()
+
+    def launch(a):
+        st = L.gca_append_frames(*a)
+        if st != 0:
+            raise gca.GcaError(st, "gca_append_frames")
+
+    for t in range(warm):  # past the window: every later launch also evicts a frame per cache
+        launch(call_args(t))
+    timed_args = [call_args(warm + i) for i in range(timed)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(20_000_000)  # ~10 ms of device time while the host enqueues below
+    e0.record(stream)
+    for a in timed_args:
+        launch(a)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / timed
+    assert all(c.check() == 0 for c in caches), "device error in the batched append"
+    bytes_per_launch = n * 6.0 * T * H * D * 2  # q, k, v in; q_rot, k, v out (K = 0: no copies)
+    for c in caches:
+        c.close()
+    return {"workload": f"{w.name}: " + workload_desc(w), "caches": n,
+            "launches_timed": timed, "frames_before_timing": warm,
+            "bytes_per_launch": bytes_per_launch, "us_per_launch": ms * 1e3,
+            "gbs": bytes_per_launch / (ms / 1e3) / 1e9}
 
 
 def run_e2e(args, w, cache, ring_host, device, stream, world):
@@ -479,6 +542,14 @@ def main():
         "gpu_launches": r["launches_per_step"] * args.steps,
         "clocks": r["clocks"],
     }
+    b = r["batched_append"]
+    if b is not None:
+        line["append_batch_roofline"] = {
+            "kernel": "gca_append_frames (one launch over 96 caches)", "bound": "hbm",
+            "achieved": b["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": b["gbs"] / pk["hbm_gbs"], "peak_kind": pk_kind,
+            **{k: v for k, v in b.items() if k != "gbs"},
+        }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, d = oracle_frames_per_s(w, [w.frames // 2, w.frames - 1])
         line["cpu_baseline"] = {

@@ -138,6 +138,21 @@ gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t w
 gca_status gca_append_frame(gca_cache* cache, int64_t frame_idx, const void* q, const void* k,
                             const void* v, void* q_rot_out, void* stream);
 
+/* gca_append_frame for n caches at once, in one kernel launch: cache caches[i] appends frame
+ * frame_idx[i] from q[i], k[i], v[i] and writes q_rot_out[i]. The caches are distinct, on one
+ * device, with the same tokens per frame and head count (other settings, e.g. window, RoPE
+ * base and page budget, may differ); 1 <= n <= 128. All arrays are host arrays of length n
+ * holding device pointers (q, k, v, q_rot_out as for gca_append_frame). Each cache's result is
+ * bit-identical to its own gca_append_frame call. All-or-nothing: the first failing check
+ * (GCA_ERR_INVALID_ARG, GCA_ERR_FRAME_ORDER, GCA_ERR_OUT_OF_PAGES) returns with nothing
+ * enqueued and no cache changed. A single 12 MB append is too short to reach HBM bandwidth;
+ * batching the appends of several caches (the layers' or streams' caches of one step) in one
+ * launch is how the append runs near copy bandwidth. The pages append per cache; the batched
+ * form is an addition of this library. */
+gca_status gca_append_frames(gca_cache* const* caches, int32_t n, const int64_t* frame_idx,
+                             const void* const* q, const void* const* k, const void* const* v,
+                             void* const* q_rot_out, void* stream);
+
 /* Attention of the last appended frame's queries over the cache (pages' compute_attention):
  * out[i][h] = softmax_j(q_rot[i][h] . k_j[h] / sqrt(D)) v_j[h] over the anchor, window and
  * trajectory keys visible at frame frame_idx (which must be the last appended frame).

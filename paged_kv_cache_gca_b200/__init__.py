@@ -17,8 +17,8 @@ __all__ = [
     "GcaError", "GcaConfig", "GcaState", "GcaAttendInfo", "lib", "library_path",
     "gca_validate_config", "gca_workspace_bytes", "gca_cache_create", "gca_append_frame",
     "gca_attend", "gca_reset", "gca_cache_destroy", "gca_check", "gca_get_state",
-    "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc", "GcaCache", "config_for",
-    "EXPORTED_SYMBOLS",
+    "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc", "gca_append_frames",
+    "GcaCache", "config_for", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -78,7 +78,7 @@ class GcaAttendInfo(ctypes.Structure):
 EXPORTED_SYMBOLS = (
     "gca_validate_config", "gca_workspace_bytes", "gca_cache_create", "gca_append_frame",
     "gca_attend", "gca_reset", "gca_cache_destroy", "gca_check", "gca_get_state",
-    "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc",
+    "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc", "gca_append_frames",
 )
 
 _lib = None
@@ -109,6 +109,7 @@ def lib():
         "gca_last_attend_info": (I32, [VP, P(GcaAttendInfo)]),
         "gca_status_string": (ctypes.c_char_p, [I32]),
         "gca_attend_noalloc": (I32, [VP, I64, VP, VP, VP]),
+        "gca_append_frames": (I32, [P(VP), I32, P(I64), P(VP), P(VP), P(VP), P(VP), VP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -156,6 +157,16 @@ def gca_attend_noalloc(handle, frame_idx, q_rot_ptr, out_ptr, stream) -> None:
     """gca_attend with its scratch in the library's fixed device array (no allocation)."""
     _ok(lib().gca_attend_noalloc(handle, frame_idx, q_rot_ptr, out_ptr, stream),
         "gca_attend_noalloc")
+
+
+def gca_append_frames(handles, frame_idx, q_ptrs, k_ptrs, v_ptrs, q_rot_ptrs, stream) -> None:
+    """One launch appending frame_idx[i] to cache handles[i] (sequences of equal length)."""
+    n = len(handles)
+    arr = lambda t, xs: (t * n)(*xs)
+    VP, I64 = ctypes.c_void_p, ctypes.c_int64
+    _ok(lib().gca_append_frames(arr(VP, handles), n, arr(I64, frame_idx), arr(VP, q_ptrs),
+                                arr(VP, k_ptrs), arr(VP, v_ptrs), arr(VP, q_rot_ptrs), stream),
+        "gca_append_frames")
 
 
 def gca_reset(handle, stream) -> None:

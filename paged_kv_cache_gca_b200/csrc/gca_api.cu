@@ -321,8 +321,11 @@ gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t w
   return GCA_OK;
 }
 
-gca_status gca_append_frame(gca_cache* c, int64_t t, const void* q, const void* k,
-                            const void* v, void* q_rot_out, void* stream) {
+namespace {
+
+// Checks one append and fills its launch parameters from the host mirror; changes nothing.
+gca_status prepare_append(gca_cache* c, int64_t t, const void* q, const void* k,
+                          const void* v, void* q_rot_out, AppendParams* out) {
   if (!c || !q || !k || !v || !q_rot_out) return GCA_ERR_INVALID_ARG;
   if (t != c->frames) return GCA_ERR_FRAME_ORDER;
   if (t >= c->cfg.max_frames) return GCA_ERR_INVALID_ARG;
@@ -338,7 +341,7 @@ gca_status gca_append_frame(gca_cache* c, int64_t t, const void* q, const void* 
   const int64_t free_count = c->free_tail - c->free_head;
   if (L.ppf + n_pop_traj > free_count) return GCA_ERR_OUT_OF_PAGES;
 
-  AppendParams p;
+  AppendParams& p = *out;
   std::memset(&p, 0, sizeof(p));
   p.q = static_cast<const uint4*>(q);
   p.k = static_cast<const uint4*>(k);
@@ -380,13 +383,58 @@ gca_status gca_append_frame(gca_cache* c, int64_t t, const void* q, const void* 
   p.n_push_items = evict ? L.ppf : 0;
   p.n_traj_items = n_pop_traj;
   p.n_aux_items = p.n_evict_items + p.n_zero_items + p.n_push_items + p.n_traj_items;
-  if (launch_append(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GCA_ERR_CUDA;
+  const int64_t block_threads = per_tok * p.tok_per_block;
+  p.n_blocks = p.n_tok_blocks + (int32_t)((p.n_aux_items + block_threads - 1) / block_threads);
+  return GCA_OK;
+}
 
-  c->free_head += L.ppf + n_pop_traj;
-  if (evict) c->free_tail += L.ppf;
-  c->traj_len += K;
-  c->traj_pages += n_pop_traj;
+// Advances the host mirror past an enqueued append.
+void commit_append(gca_cache* c, const AppendParams& p) {
+  c->free_head += c->lay.ppf + p.n_pop_traj;
+  if (p.evict_frame >= 0) c->free_tail += c->lay.ppf;
+  c->traj_len += p.K;
+  c->traj_pages += p.n_pop_traj;
   c->frames += 1;
+}
+
+}  // namespace
+
+gca_status gca_append_frame(gca_cache* c, int64_t t, const void* q, const void* k,
+                            const void* v, void* q_rot_out, void* stream) {
+  AppendParams p;
+  const gca_status st = prepare_append(c, t, q, k, v, q_rot_out, &p);
+  if (st != GCA_OK) return st;
+  if (launch_append(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GCA_ERR_CUDA;
+  commit_append(c, p);
+  return GCA_OK;
+}
+
+gca_status gca_append_frames(gca_cache* const* caches, int32_t n, const int64_t* frame_idx,
+                             const void* const* q, const void* const* k, const void* const* v,
+                             void* const* q_rot_out, void* stream) {
+  if (!caches || !frame_idx || !q || !k || !v || !q_rot_out) return GCA_ERR_INVALID_ARG;
+  if (n < 1 || n > kMaxAppendBatch) return GCA_ERR_INVALID_ARG;
+  static thread_local AppendBatch b;  // ~30 KB: kept off the stack
+  b.n = n;
+  b.max_blocks = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    gca_cache* c = caches[i];
+    if (!c) return GCA_ERR_INVALID_ARG;
+    for (int32_t j = 0; j < i; ++j) {
+      if (caches[j] == c) return GCA_ERR_INVALID_ARG;  // one frame per cache per launch
+    }
+    if (c->device != caches[0]->device || c->lay.T != caches[0]->lay.T ||
+        c->cfg.num_heads != caches[0]->cfg.num_heads) {
+      return GCA_ERR_INVALID_ARG;
+    }
+    const gca_status st = prepare_append(c, frame_idx[i], q[i], k[i], v[i], q_rot_out[i], &b.p[i]);
+    if (st != GCA_OK) return st;
+    b.max_blocks = std::max(b.max_blocks, b.p[i].n_blocks);
+  }
+  if (launch_append_batch(b, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    return GCA_ERR_CUDA;
+  }
+  for (int32_t i = 0; i < n; ++i) commit_append(caches[i], b.p[i]);
   return GCA_OK;
 }
 

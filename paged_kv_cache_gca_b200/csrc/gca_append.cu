@@ -120,16 +120,17 @@ __device__ __forceinline__ uint32_t rotate_word(uint32_t w, float2 cs) {
 
 __device__ __forceinline__ int wrap(int pos, int n) { return pos >= n ? pos - n : pos; }
 
-// Token part: block (8 chunks, H heads, tok_per_block tokens); one thread = one 16-byte chunk
-// (8 dims) of one (token, head). Auxiliary part (blocks after n_tok_blocks): eviction copies,
-// zero fill of a fresh trajectory page, free-list pushes, trajectory page records.
-__global__ void __launch_bounds__(1024) append_kernel(const AppendParams p) {
+// Block bx of one cache's append. Token part: block (8 chunks, H heads, tok_per_block tokens);
+// one thread = one 16-byte chunk (8 dims) of one (token, head). Auxiliary part (blocks after
+// n_tok_blocks): eviction copies, zero fill of a fresh trajectory page, free-list pushes,
+// trajectory page records.
+__device__ __forceinline__ void append_block(const AppendParams& p, const int bx) {
   const int H = p.H;
-  if (blockIdx.x < (unsigned)p.n_tok_blocks) {
+  if (bx < p.n_tok_blocks) {
     // ---- a1 + a2
     const int c = threadIdx.x;
     const int h = threadIdx.y;
-    const int i = blockIdx.x * p.tok_per_block + threadIdx.z;
+    const int i = bx * p.tok_per_block + threadIdx.z;
     if (i >= p.ppf * kPageSize) return;
     const int page = p.free_ring[wrap(p.head_pos + i / kPageSize, p.num_pages)];
     if (page < 0 || page >= p.num_pages) {
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(1024) append_kernel(const AppendParams p) {
 
   const int block_threads = 8 * H * p.tok_per_block;
   const int lin = threadIdx.x + 8 * (threadIdx.y + H * threadIdx.z);
-  const int64_t idx = (int64_t)(blockIdx.x - p.n_tok_blocks) * block_threads + lin;
+  const int64_t idx = (int64_t)(bx - p.n_tok_blocks) * block_threads + lin;
   if (idx >= p.n_aux_items) return;
   const int64_t e_ev = p.n_evict_items;
   const int64_t e_zero = e_ev + p.n_zero_items;
@@ -240,6 +241,15 @@ __global__ void __launch_bounds__(1024) append_kernel(const AppendParams p) {
   p.traj_pages[p.traj_pages_before + k] = p.free_ring[wrap(first_new + k, p.num_pages)];
 }
 
+__global__ void __launch_bounds__(1024) append_kernel(const AppendParams p) {
+  append_block(p, (int)blockIdx.x);
+}
+
+__global__ void __launch_bounds__(1024) append_batch_kernel(const __grid_constant__ AppendBatch b) {
+  const AppendParams& p = b.p[blockIdx.y];
+  if ((int)blockIdx.x < p.n_blocks) append_block(p, (int)blockIdx.x);
+}
+
 }  // namespace
 
 cudaError_t launch_init(const InitParams& p, cudaStream_t s) {
@@ -265,10 +275,14 @@ cudaError_t launch_reset(int32_t* free_ring, const int32_t* init_free, uint32_t*
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
-  const int64_t block_threads = 8LL * p.H * p.tok_per_block;
-  const int64_t aux_blocks = (p.n_aux_items + block_threads - 1) / block_threads;
   const dim3 block(8, p.H, p.tok_per_block);
-  append_kernel<<<(unsigned)(p.n_tok_blocks + aux_blocks), block, 0, s>>>(p);
+  append_kernel<<<(unsigned)p.n_blocks, block, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_batch(const AppendBatch& b, cudaStream_t s) {
+  const dim3 block(8, b.p[0].H, b.p[0].tok_per_block);
+  append_batch_kernel<<<dim3((unsigned)b.max_blocks, (unsigned)b.n), block, 0, s>>>(b);
   return cudaGetLastError();
 }
 

@@ -54,6 +54,19 @@
 //                  spins with __nanosleep(n) between polls.
 //   GCA_TURN_EARLY the turn passes to the other warpgroup this many 32-column chunks before
 //                  this one's exponentials are done.
+//   GCA_MMA_SPIN   1: the MMA-issuing threads spin on their barriers; 0: they sleep in try_wait.
+//   GCA_SM_SPIN    1: the softmax warps spin on S, slot counts and P V completion; 0: sleep.
+//   GCA_LATE_PV    1: the softmax waits for P V of the previous tile only before it stores the
+//                  new P (after its exponentials); 0: before its turn.
+#ifndef GCA_MMA_SPIN
+#define GCA_MMA_SPIN 1
+#endif
+#ifndef GCA_SM_SPIN
+#define GCA_SM_SPIN 0
+#endif
+#ifndef GCA_LATE_PV
+#define GCA_LATE_PV 0
+#endif
 //   GCA_TURNS      1: the two softmax warpgroups take turns for the exponentials; 0: both
 //                  compute them whenever their scores are ready.
 #ifndef GCA_TURNS
@@ -80,7 +93,7 @@ namespace gca {
 #if GCA_TRACE
 // Event timestamps (clock64) of the first tiles of CTAs 0 and 1, for pipeline studies; read
 // back with gca_debug_trace in builds with -DGCA_TRACE=1.
-__device__ long long g_trace[2][64][16];
+__device__ long long g_trace[2][64][32];
 #define TRACE(slot, tile)                                                                   \
   do {                                                                                      \
     if (blockIdx.x < 2 && (tile) < 64) g_trace[blockIdx.x][(tile)][(slot)] = clock64();     \
@@ -214,15 +227,15 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, Share
   }
 }
 
-// Spinning variant (no hardware suspend) for short, latency-critical hand-overs.
+// Spinning variant (no hardware suspend) for short, latency-critical hand-overs: a thread
+// suspended in try_wait resumes some hundreds of cycles after the phase completes.
+template <int kBackoffNs = 0>
 __device__ __forceinline__ bool spin_phase(uint64_t* bar, uint32_t parity, Shared* sh,
                                            uint32_t* err) {
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer();
   for (uint32_t i = 1;; ++i) {
-#if GCA_TURN_SPIN >= 2
-    __nanosleep(GCA_TURN_SPIN);  // back off: polls are shared-memory (MIO) instructions
-#endif
+    if (kBackoffNs > 0) __nanosleep(kBackoffNs);
     if (mbar_test_wait(bar, parity)) return true;
     if ((i & 255u) == 0u) {
       if (sh->abort_flag) return false;
@@ -235,11 +248,31 @@ __device__ __forceinline__ bool spin_phase(uint64_t* bar, uint32_t parity, Share
   }
 }
 
+// The MMA issuers' waits: on the critical path from "P ready" to "P V issued".
+__device__ __forceinline__ bool mma_wait(uint64_t* bar, uint32_t parity, Shared* sh,
+                                         uint32_t* err) {
+#if GCA_MMA_SPIN
+  return spin_phase(bar, parity, sh, err);
+#else
+  return wait_phase(bar, parity, sh, err);
+#endif
+}
+
 // Every lane of the warp waits; the result is agreed across the warp so that warp-collective
 // instructions after it never run with diverged lanes.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Shared* sh,
                                           uint32_t* err, bool drain = false) {
   return __all_sync(0xffffffffu, wait_phase(bar, parity, sh, err, drain));
+}
+
+// The softmax warps' waits for S, the key-slot counts and P V completion.
+__device__ __forceinline__ bool sm_wait(uint64_t* bar, uint32_t parity, Shared* sh,
+                                        uint32_t* err) {
+#if GCA_SM_SPIN
+  return __all_sync(0xffffffffu, spin_phase(bar, parity, sh, err));
+#else
+  return warp_wait(bar, parity, sh, err);
+#endif
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -564,10 +597,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = j0; j <= j1; ++j) {
           if (j < j1) {
             const int ks = it % kKStages;
-            if (!wait_phase(&sh.k_full[ks], (it / kKStages) & 1u, &sh, p.err)) { ok = false; break; }
-            if (j > j0 && !wait_phase(&sh.s_free[qq], (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
+            if (!mma_wait(&sh.k_full[ks], (it / kKStages) & 1u, &sh, p.err)) { ok = false; break; }
+            if (j > j0 && !mma_wait(&sh.s_free[qq], (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
             tc_fence_after();
-            if (qq == 0) TRACE(2, it);
+            TRACE(qq ? 20 : 2, it);
             const uint64_t k_desc = sw128_desc(smem_addr(k_smem + ks * kTileBytes), 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < kHeadDim / 16; ++kk) {
@@ -576,15 +609,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mma_commit(&sh.s_full[qq]);
             mma_commit(&sh.k_empty[ks]);
-            if (qq == 0) TRACE(3, it);
+            TRACE(qq ? 21 : 3, it);
           }
           if (j > j0) {
             const uint32_t pit = it - 1;  // tile j-1
             const int vs = pit % kVStages;
-            if (!wait_phase(&sh.p_full[qq], pit & 1u, &sh, p.err)) { ok = false; break; }
-            if (!wait_phase(&sh.v_full[vs], (pit / kVStages) & 1u, &sh, p.err)) { ok = false; break; }
+            if (!mma_wait(&sh.p_full[qq], pit & 1u, &sh, p.err)) { ok = false; break; }
+            if (!mma_wait(&sh.v_full[vs], (pit / kVStages) & 1u, &sh, p.err)) { ok = false; break; }
             tc_fence_after();
-            if (qq == 0) TRACE(4, pit);
+            TRACE(qq ? 22 : 4, pit);
             const uint64_t v_desc = sw128_desc(smem_addr(v_smem + vs * kTileBytes), 16384, 1024);
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk) {
@@ -594,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mma_commit(&sh.pv_done[qq]);
             mma_commit(&sh.v_empty[vs]);
-            if (qq == 0) TRACE(5, pit);
+            TRACE(qq ? 23 : 5, pit);
           }
           if (j < j1) ++it;
         }
@@ -642,10 +675,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m_run = -INFINITY;  // running row max, log2 units (scaled)
       float l_run = 0.f;        // running row sum relative to m_run
       for (int j = j0; j < j1; ++j, ++it) {
-        if (!warp_wait(&sh.s_full[qq], it & 1u, &sh, p.err)) { ok = false; break; }
-        if (!warp_wait(&sh.lens_full[it & 3], (it >> 2) & 1u, &sh, p.err)) { ok = false; break; }
+        if (!sm_wait(&sh.s_full[qq], it & 1u, &sh, p.err)) { ok = false; break; }
+        if (r == 0) TRACE(16 + qq, it);
+        if (!sm_wait(&sh.lens_full[it & 3], (it >> 2) & 1u, &sh, p.err)) { ok = false; break; }
         const uint64_t lens = sh.lens[it & 3];
-        if (r == 0 && qq == 0) TRACE(6, it);
+        if (r == 0) TRACE(6 + 5 * qq, it);
         tc_fence_after();
         float sv[kTileK];
         tmem_ld128(t_row + kColS, sv);
@@ -685,48 +719,63 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_new = tile_max;
           alpha = ex2(m_run - m_new);
         }
-        if (j > j0) {
+        if (!GCA_LATE_PV && j > j0) {
           // P V of the previous tile must be done before P is overwritten or O rescaled
-          if (!warp_wait(&sh.pv_done[qq], (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
+          if (!sm_wait(&sh.pv_done[qq], (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
           tc_fence_after();
         }
+        if (r == 0) TRACE(7 + 5 * qq, it);
         // P = 2^(s*c - m), inside this warpgroup's turn on MUFU: scale-subtract, exponentials,
         // bf16 packing, row sum and TMEM stores, 32 columns at a time. The turn passes to the
         // other warpgroup GCA_TURN_EARLY chunks before the end so that its first exponentials
         // queue behind this group's last ones.
 #if GCA_TURNS && GCA_TURN_SPIN
-        if (!__all_sync(0xffffffffu, spin_phase(&sh.turn[qq], turns & 1u, &sh, p.err))) {
+        if (!__all_sync(0xffffffffu, spin_phase<(GCA_TURN_SPIN >= 2 ? GCA_TURN_SPIN : 0)>(&sh.turn[qq], turns & 1u, &sh, p.err))) {
           ok = false;
           break;
         }
 #elif GCA_TURNS
         if (!warp_wait(&sh.turn[qq], turns & 1u, &sh, p.err)) { ok = false; break; }
 #endif
-        if (r == 0 && qq == 0) TRACE(7, it);
+        if (r == 0) TRACE(8 + 5 * qq, it);
         const float neg_m = -m_new;
 #pragma unroll
         for (int e = 0; e < kTileK; ++e) sv[e] = fmaf(sv[e], p.scale_log2, neg_m);
         float rs[8];
 #pragma unroll
         for (int a = 0; a < 8; ++a) rs[a] = 0.f;
+        uint32_t pk[kTileK / 2];
 #pragma unroll
         for (int chunk = 0; chunk < kTileK / 32; ++chunk) {
-          uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int e = 32 * chunk + 2 * c;
             const bool poly = c < GCA_POLY_PAIRS;
             const float e0 = poly ? exp2_poly(sv[e]) : ex2(sv[e]);
             const float e1 = poly ? exp2_poly(sv[e + 1]) : ex2(sv[e + 1]);
-            pk[c] = pack_bf2(e0, e1);
+            pk[16 * chunk + c] = pack_bf2(e0, e1);
             rs[2 * (c & 3)] += e0;
             rs[2 * (c & 3) + 1] += e1;
           }
-          tmem_st16(t_row + kColP + 16 * chunk, reinterpret_cast<const float*>(pk));
+          if (!GCA_LATE_PV) {
+            tmem_st16(t_row + kColP + 16 * chunk, reinterpret_cast<const float*>(pk + 16 * chunk));
+          }
           if (GCA_TURNS && chunk == kTileK / 32 - 1 - GCA_TURN_EARLY) mbar_arrive(&sh.turn[qq ^ 1]);
         }
         ++turns;
-        if (r == 0 && qq == 0) TRACE(8, it);
+        if (r == 0) TRACE(9 + 5 * qq, it);
+        if (GCA_LATE_PV) {
+          // P V of the previous tile must be done before P is overwritten or O rescaled
+          if (j > j0) {
+            if (!sm_wait(&sh.pv_done[qq], (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
+            tc_fence_after();
+          }
+          if (r == 0) TRACE(18 + qq, it);
+#pragma unroll
+          for (int chunk = 0; chunk < kTileK / 32; ++chunk) {
+            tmem_st16(t_row + kColP + 16 * chunk, reinterpret_cast<const float*>(pk + 16 * chunk));
+          }
+        }
         // Lazy rescale of O (rare): after the scores are dead, before P V(j) is issued.
         if (j > j0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
@@ -745,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sh.p_full[qq]);
-        if (r == 0 && qq == 0) TRACE(9, it);
+        if (r == 0) TRACE(10 + 5 * qq, it);
       }
       if (!ok) break;
 
@@ -792,6 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                  "r"(kTmemCols));
   }
 }
+
 
 // Merges the partial records of every split (head, query tile): weights 2^(m_s - M),
 // M = max_s m_s. Two threads per query row, 32 output columns each.
@@ -866,6 +916,7 @@ cudaError_t launch_combine(const AttnParams& p, cudaStream_t s) {
   combine_kernel<<<p.units, kCombineThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
+
 
 }  // namespace gca
 

@@ -22,6 +22,7 @@ constexpr int kTileK = 128;     // keys per attention tile (8 pages)
 constexpr int kPagesPerTile = kTileK / kPageSize;
 constexpr int kMaxGrid = 512;   // attention CTAs per launch (sizes the split buffers)
 constexpr size_t kAlign = 1024;
+constexpr int kMaxAppendBatch = 128;  // caches per batched append launch (kernel-parameter bound)
 
 // Byte offsets of every region inside the caller's workspace.
 struct Layout {
@@ -97,8 +98,18 @@ struct AppendParams {
   // launch shape: token blocks of (8 chunks, H heads, tok_per_block tokens) threads, then
   // blocks of kAuxThreads for the eviction items
   int32_t tok_per_block, n_tok_blocks;
+  int32_t n_blocks;  // token blocks + auxiliary blocks
   int64_t n_evict_items, n_zero_items, n_push_items, n_traj_items, n_aux_items;
 };
+
+// One frame appended to each of n caches of the same shape (T, H), in one launch: block
+// (x, y) is block x of cache y's own append.
+struct AppendBatch {
+  int32_t n;
+  int32_t max_blocks;
+  AppendParams p[kMaxAppendBatch];
+};
+static_assert(sizeof(AppendBatch) <= 32764, "kernel parameter space");
 
 struct AttnParams {
   const uint4* q;        // rotated queries [T][H][64] bf16
@@ -131,6 +142,7 @@ cudaError_t launch_check_perm(int32_t* seen, uint32_t* err, int32_t n, cudaStrea
 cudaError_t launch_reset(int32_t* free_ring, const int32_t* init_free, uint32_t* err,
                          int32_t n, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+cudaError_t launch_append_batch(const AppendBatch& b, cudaStream_t s);
 cudaError_t attn_prepare(int* ctas_per_sm);  // sets kernel attributes, reports occupancy
 cudaError_t launch_attn(const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
                         cudaStream_t s);

@@ -4,6 +4,11 @@ For profilers: the appends of frames 0..t run first (cheap kernels), then exactl
 attention calls at frame t, so a capture can select them with few launches before them.
 
     python -m paged_kv_cache_gca_b200.profile_frame --workload w16_320 --frame 319 --repeat 1
+
+With --batch N it instead creates N caches of the workload and runs --frame + 1 batched appends
+(gca_append_frames over all N caches; frame of cache c at step t: ring slot (N t + c) mod R):
+
+    python -m paged_kv_cache_gca_b200.profile_frame --workload stack24x4 --batch 16 --frame 15
 """
 import argparse
 import os
@@ -24,7 +29,10 @@ def main():
     ap.add_argument("--workload", default="w16_320")
     ap.add_argument("--frame", type=int, default=-1)
     ap.add_argument("--repeat", type=int, default=1)
+    ap.add_argument("--batch", type=int, default=0)
     args = ap.parse_args()
+    if args.batch > 0:
+        return batched(args)
     w = gi.workload(args.workload)
     t_last = w.frames - 1 if args.frame < 0 else args.frame
     T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
@@ -42,6 +50,27 @@ def main():
     inf = cache.attend_info()
     print(f"{w.name} t={t_last}: Nk={inf.visible_keys} grid={inf.grid} split={inf.split} "
           f"status={status}")
+    sys.exit(0 if status == 0 else 1)
+
+
+def batched(args):
+    w = gi.workload(args.workload)
+    n = args.batch
+    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    ring = gi.draw_ring(w).cuda()
+    R = ring.shape[0]
+    caches = [gca.GcaCache(gca.config_for(w, gi.rope_base_for_layer(w, c % w.num_layers)))
+              for c in range(n)]
+    q_rot = [torch.empty((T, H, D), dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    stream = torch.cuda.current_stream().cuda_stream
+    for t in range(args.frame + 1):
+        f = [ring[(n * t + c) % R] for c in range(n)]
+        gca.gca_append_frames([c.handle for c in caches], [t] * n, [x[0].data_ptr() for x in f],
+                              [x[1].data_ptr() for x in f], [x[2].data_ptr() for x in f],
+                              [x.data_ptr() for x in q_rot], stream)
+    torch.cuda.synchronize()
+    status = max(c.check() for c in caches)
+    print(f"{w.name} x{n}: {args.frame + 1} batched appends, status={status}")
     sys.exit(0 if status == 0 else 1)
 
 

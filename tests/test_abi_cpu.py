@@ -101,3 +101,13 @@ def test_create_rejects_bad_arguments_before_touching_cuda(L):
     assert L.gca_reset(None, None) == -1
     assert L.gca_check(None) == -1
     assert L.gca_cache_destroy(None) == 0
+    # batched append: empty or oversized batch, null arrays, null cache
+    VP, I64 = ctypes.c_void_p, ctypes.c_int64
+    one = (VP * 1)(1)
+    idx = (I64 * 1)(0)
+    nul = (VP * 1)(None)
+    assert L.gca_append_frames(one, 0, idx, one, one, one, one, None) == -1
+    assert L.gca_append_frames(one, 129, idx, one, one, one, one, None) == -1
+    assert L.gca_append_frames(None, 1, idx, one, one, one, one, None) == -1
+    assert L.gca_append_frames(one, 1, None, one, one, one, one, None) == -1
+    assert L.gca_append_frames(nul, 1, idx, one, one, one, one, None) == -1
