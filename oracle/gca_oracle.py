@@ -40,6 +40,15 @@ Readings where the pages are silent (each is listed in the design notes):
      page whenever the tail page is full (trajectory pages are dense and never freed), and
      finally pushes the evicted frame's pages to the tail in row order. Anchor pages are
      never freed. Reset restores the initial order.
+  R7 keyframe-only caching [GCT, FlashInferBlock `skip_append`; Streaming Inference API
+     `keyframe_interval`]: video frame g is a keyframe when g % N == 0. Cache frames ("slots")
+     count the kept frames; a keyframe takes the next slot with the normal append -> evict ->
+     attend. A non-keyframe takes the next slot transiently: append (pages popped, nothing
+     evicted) -> attend -> roll back (its pages return to the free-list head in reverse order,
+     which restores the allocator exactly). With no eviction before its attention, a transient
+     frame at slot s sees the anchors, window slots max(A, s-W)..s (up to W+1 frames, itself
+     included) and the kept tokens of slots A..s-W-1. The RoPE time position of a slot is the
+     global index g of the video frame it holds [GCT, 3D RoPE]; without keyframes g = slot.
 """
 from __future__ import annotations
 
@@ -58,6 +67,7 @@ __all__ = [
     "pool_frames",
     "visible_keys",
     "visible_key_count",
+    "keyframe_stream",
     "softmax_attention",
     "FifoPages",
     "CacheBook",
@@ -135,28 +145,29 @@ def kept_token_indices(num_special: int, num_patches: int, keep: int):
     return list(range(num_special)) + [num_special + j * stride for j in range(extra)]
 
 
-def pool_frames(t: int, A: int, W: int):
-    """(anchor frames, window frames, evicted frames) visible at step t (reading R3)."""
+def pool_frames(t: int, A: int, W: int, transient: bool = False):
+    """(anchor frames, window frames, evicted frames) visible at step t (reading R3); for a
+    transient (non-keyframe) frame at slot t, nothing was evicted before its attention (R7)."""
     if t < A:
         return list(range(t + 1)), [], []
     anchor = list(range(A))
-    w0 = max(A, t - W + 1)
+    w0 = max(A, t - W + (0 if transient else 1))
     window = list(range(w0, t + 1))
     evicted = list(range(A, w0))
     return anchor, window, evicted
 
 
-def visible_keys(t: int, A: int, W: int, T: int, kept):
+def visible_keys(t: int, A: int, W: int, T: int, kept, transient: bool = False):
     """Pool-ordered list of (frame, token) keys that frame t's queries see."""
-    anchor, window, evicted = pool_frames(t, A, W)
+    anchor, window, evicted = pool_frames(t, A, W, transient)
     keys = [(f, i) for f in anchor for i in range(T)]
     keys += [(f, i) for f in window for i in range(T)]
     keys += [(f, i) for f in evicted for i in kept]
     return keys
 
 
-def visible_key_count(t: int, A: int, W: int, T: int, K: int) -> int:
-    anchor, window, evicted = pool_frames(t, A, W)
+def visible_key_count(t: int, A: int, W: int, T: int, K: int, transient: bool = False) -> int:
+    anchor, window, evicted = pool_frames(t, A, W, transient)
     return (len(anchor) + len(window)) * T + len(evicted) * K
 
 
@@ -195,6 +206,10 @@ class FifoPages:
     def reset(self) -> None:
         self.free = deque(self.initial)
 
+    def unpop(self, page: int) -> None:
+        """Return a page to the head (undo of the last pop)."""
+        self.free.appendleft(page)
+
 
 class CacheBook:
     """Integer state of one cache: page rows per frame, slot map, trajectory pages.
@@ -220,6 +235,7 @@ class CacheBook:
         self.traj_tokens = []  # (frame, token) per trajectory slot, in order
         self.frames = 0
         self.slot_map = []
+        self.transient = False  # the last append was a non-keyframe awaiting rollback (R7)
 
     @property
     def traj_len(self):
@@ -228,17 +244,18 @@ class CacheBook:
     def pages_in_use(self):
         return sum(len(r) for r in self.frame_pages.values()) + len(self.traj_pages)
 
-    def append(self, t: int):
-        if t != self.frames:
-            raise ValueError("frames must be appended in order")
+    def append(self, t: int, transient: bool = False):
+        if t != self.frames or self.transient:
+            raise ValueError("frames must be appended in order (a transient frame first rolls back)")
         # 1. the new frame's pages, popped in order
         row = [self.alloc.pop() for _ in range(self.ppf)]
         self.frame_pages[t] = row
         self.all_rows[t] = row
         self.slot_map = [row[i // self.ps] * self.ps + i % self.ps for i in range(self.T)]
-        # 2. eviction of the frame that left the window
+        self.transient = transient
+        # 2. eviction of the frame that left the window (none for a transient frame, R7)
         e = t - self.W
-        if e >= self.A:
+        if e >= self.A and not transient:
             for i in self.kept:
                 if self.traj_len % self.ps == 0:
                     self.traj_pages.append(self.alloc.pop())
@@ -246,6 +263,18 @@ class CacheBook:
             for p in self.frame_pages.pop(e):
                 self.alloc.push(p)
         self.frames += 1
+
+    def rollback(self, t: int):
+        """Undo the transient append of frame t: its pages go back to the free-list head in
+        reverse order, so the free list is exactly what it was before the append (R7)."""
+        if not self.transient or t != self.frames - 1:
+            raise ValueError("only a transient last frame rolls back")
+        row = self.frame_pages.pop(t)
+        self.all_rows.pop(t)
+        for p in reversed(row):
+            self.alloc.unpop(p)
+        self.frames -= 1
+        self.transient = False
 
     def location_of(self, frame: int, token: int):
         """(page, slot) that holds a live frame's token."""
@@ -263,9 +292,12 @@ class CacheBook:
 class GcaOracle:
     """fp64 oracle of one GCA cache fed by a seeded synthetic stream.
 
-    `frame_source(t)` returns the bf16 (q, k, v) tensors [T, H, D] of frame t (torch or
-    numpy); they are widened exactly. `slot_of(t)` names the distinct input frame that frame t
+    `frame_source(g)` returns the bf16 (q, k, v) tensors [T, H, D] of video frame g (torch or
+    numpy); they are widened exactly. `slot_of(g)` names the distinct input frame that frame g
     reuses (identity by default), so long streams keep a bounded set of raw frames in memory.
+    Cache frame (slot) t holds video frame gidx[t]: t itself unless `append` was given another
+    global index (keyframe streams, R7); its RoPE time position and its inputs are those of
+    gidx[t].
     """
 
     def __init__(self, *, num_heads, head_dim, page_size, grid_h, grid_w, num_special,
@@ -291,12 +323,17 @@ class GcaOracle:
                               initial_free=initial_free)
         self._raw = {}  # slot -> (q, k, v) as float32 arrays (exact copies of bf16)
         self._pos = token_positions(0, self.S, self.gh, self.gw)
+        self.gidx = {}  # cache frame -> global (video) frame index, when not the identity
+
+    def global_index(self, t):
+        return self.gidx.get(int(t), int(t))
 
     # inputs ---------------------------------------------------------------------------
     def raw32(self, t):
-        slot = self.slot_of(t)
+        g = self.global_index(t)
+        slot = self.slot_of(g)
         if slot not in self._raw:
-            q, k, v = self.source(t)
+            q, k, v = self.source(g)
             self._raw[slot] = tuple(_to_f32(x) for x in (q, k, v))
         return self._raw[slot]
 
@@ -308,7 +345,7 @@ class GcaOracle:
         frames = np.asarray(frames, dtype=np.int64)
         tokens = np.asarray(tokens, dtype=np.int64)
         pos = self._pos[tokens].copy()
-        pos[:, 0] = frames
+        pos[:, 0] = [self.global_index(f) for f in frames] if self.gidx else frames
         return pos
 
     def q_rot(self, t, rows=None):
@@ -324,15 +361,28 @@ class GcaOracle:
         return rotate_pairs(k, ang)
 
     # bookkeeping ----------------------------------------------------------------------
-    def append(self, t):
-        self.book.append(t)
+    def append(self, t, g=None, transient=False):
+        """Append cache frame t holding video frame g (default t); transient: a non-keyframe
+        that will roll back (R7)."""
+        self.book.append(t, transient)
+        if g is None or g == t:
+            self.gidx.pop(t, None)
+        else:
+            self.gidx[t] = int(g)
+
+    def rollback(self, t):
+        self.book.rollback(t)
+        self.gidx.pop(t, None)
+
+    def _transient(self, t):
+        return self.book.transient and t == self.book.frames - 1
 
     def visible(self, t):
-        return visible_keys(t, self.A, self.W, self.T, self.kept)
+        return visible_keys(t, self.A, self.W, self.T, self.kept, self._transient(t))
 
     def key_index(self, t):
         """(frames, tokens) int arrays of the keys frame t sees, in pool order."""
-        anchor, window, evicted = pool_frames(t, self.A, self.W)
+        anchor, window, evicted = pool_frames(t, self.A, self.W, self._transient(t))
         full = np.asarray(anchor + window, dtype=np.int64)
         fr = [np.repeat(full, self.T)]
         tk = [np.tile(np.arange(self.T, dtype=np.int64), len(full))]
@@ -350,7 +400,7 @@ class GcaOracle:
             angles = rope_angles(self.positions(frames, tokens), self.D, self.base)
         k = np.empty((len(frames), self.D), dtype=np.float64)
         v = np.empty((len(frames), self.D), dtype=np.float64)
-        slots = np.asarray([self.slot_of(int(f)) for f in frames])
+        slots = np.asarray([self.slot_of(self.global_index(f)) for f in frames])
         for s in np.unique(slots):
             sel = np.nonzero(slots == s)[0]
             f0 = int(frames[sel[0]])
@@ -370,6 +420,24 @@ class GcaOracle:
             k, v = self.gather_head(t, h, frames, tokens, angles)
             out[:, h, :] = softmax_attention(qr[:, h, :], k, v)
         return out
+
+
+def keyframe_stream(oracle: GcaOracle, frames: int, interval: int, on_frame=None):
+    """Streams video frames 0..frames-1 keeping every `interval`-th one (R7). After each
+    frame's append, `on_frame(g, slot, keyframe)` runs (the frame's attention happens there);
+    a non-keyframe then rolls back. Returns the slots of the keyframes."""
+    kept = []
+    for g in range(frames):
+        slot = oracle.book.frames
+        key = g % interval == 0
+        oracle.append(slot, g, transient=not key)
+        if on_frame is not None:
+            on_frame(g, slot, key)
+        if key:
+            kept.append(slot)
+        else:
+            oracle.rollback(slot)
+    return kept
 
 
 def _to_f32(x):
