@@ -87,7 +87,7 @@ typedef struct {
   int32_t pages_per_frame;
   int32_t pages_in_use;
   uint32_t device_error; /* last value read by gca_check() */
-  int32_t reserved;
+  int32_t transient;     /* 1 while the last append is a non-keyframe awaiting rollback */
   void* k_pool;          /* bf16 [num_pages][H][page_size][D]: rotated keys */
   void* v_pool;          /* bf16 [num_pages][H][page_size][D]: values */
   int32_t* free_ring;    /* int32 [num_pages] */
@@ -137,6 +137,36 @@ gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t w
  * mirrored counts: GCA_ERR_OUT_OF_PAGES returns with nothing enqueued. */
 gca_status gca_append_frame(gca_cache* cache, int64_t frame_idx, const void* q, const void* k,
                             const void* v, void* q_rot_out, void* stream);
+
+/* Flags of gca_append_frame_ex. */
+enum {
+  /* A non-keyframe (pages' skip_append path, keyframe-only caching): the frame's K/V are
+   * appended and it may be attended, but nothing is evicted, and gca_rollback_last_frame must
+   * follow before the next append. While it is pending, gca_attend of this frame sees the
+   * anchors, the window frames still cached plus this one (up to W+1 frames) and the
+   * trajectory. */
+  GCA_APPEND_TRANSIENT = 1
+};
+
+/* gca_append_frame with an explicit RoPE time position and flags. frame_idx is the cache
+ * frame (the number of frames kept so far: non-keyframes do not count once rolled back);
+ * rope_frame is the global index of the video frame (the time position of its 3D RoPE;
+ * 0 <= rope_frame < max_frames). gca_append_frame(c, t, ...) is
+ * gca_append_frame_ex(c, t, t, 0, ...). Errors as gca_append_frame, and GCA_ERR_FRAME_ORDER
+ * while a transient frame awaits rollback; GCA_ERR_INVALID_ARG for unknown flags. */
+gca_status gca_append_frame_ex(gca_cache* cache, int64_t frame_idx, int64_t rope_frame,
+                               uint32_t flags, const void* q, const void* k, const void* v,
+                               void* q_rot_out, void* stream);
+
+/* Undoes the transient append of frame frame_idx (pages' rollback_last_frame): the frame's
+ * pages return to the head of the free list in reverse order, which restores the allocator
+ * exactly, and the frame count goes back to frame_idx. Host bookkeeping only: nothing is
+ * enqueued (the device ring still holds the page ids at those positions; the pages' contents
+ * are left as they are and are overwritten when popped again). Work already enqueued that
+ * reads the frame (its gca_attend) must be ordered before the next append, which is the case
+ * on one stream. GCA_ERR_FRAME_ORDER unless the last append was transient and was frame
+ * frame_idx. `stream` is unused. */
+gca_status gca_rollback_last_frame(gca_cache* cache, int64_t frame_idx, void* stream);
 
 /* gca_append_frame for n caches at once, in one kernel launch: cache caches[i] appends frame
  * frame_idx[i] from q[i], k[i], v[i] and writes q_rot_out[i]. The caches are distinct, on one

@@ -40,7 +40,7 @@ Readings where the pages are silent (each is listed in the design notes):
      page whenever the tail page is full (trajectory pages are dense and never freed), and
      finally pushes the evicted frame's pages to the tail in row order. Anchor pages are
      never freed. Reset restores the initial order.
-  R7 keyframe-only caching [GCT, FlashInferBlock `skip_append`; Streaming Inference API
+  R11 keyframe-only caching [GCT, FlashInferBlock `skip_append`; Streaming Inference API
      `keyframe_interval`]: video frame g is a keyframe when g % N == 0. Cache frames ("slots")
      count the kept frames; a keyframe takes the next slot with the normal append -> evict ->
      attend. A non-keyframe takes the next slot transiently: append (pages popped, nothing
@@ -147,7 +147,7 @@ def kept_token_indices(num_special: int, num_patches: int, keep: int):
 
 def pool_frames(t: int, A: int, W: int, transient: bool = False):
     """(anchor frames, window frames, evicted frames) visible at step t (reading R3); for a
-    transient (non-keyframe) frame at slot t, nothing was evicted before its attention (R7)."""
+    transient (non-keyframe) frame at slot t, nothing was evicted before its attention (R11)."""
     if t < A:
         return list(range(t + 1)), [], []
     anchor = list(range(A))
@@ -235,7 +235,7 @@ class CacheBook:
         self.traj_tokens = []  # (frame, token) per trajectory slot, in order
         self.frames = 0
         self.slot_map = []
-        self.transient = False  # the last append was a non-keyframe awaiting rollback (R7)
+        self.transient = False  # the last append was a non-keyframe awaiting rollback (R11)
 
     @property
     def traj_len(self):
@@ -253,7 +253,7 @@ class CacheBook:
         self.all_rows[t] = row
         self.slot_map = [row[i // self.ps] * self.ps + i % self.ps for i in range(self.T)]
         self.transient = transient
-        # 2. eviction of the frame that left the window (none for a transient frame, R7)
+        # 2. eviction of the frame that left the window (none for a transient frame, R11)
         e = t - self.W
         if e >= self.A and not transient:
             for i in self.kept:
@@ -266,7 +266,7 @@ class CacheBook:
 
     def rollback(self, t: int):
         """Undo the transient append of frame t: its pages go back to the free-list head in
-        reverse order, so the free list is exactly what it was before the append (R7)."""
+        reverse order, so the free list is exactly what it was before the append (R11)."""
         if not self.transient or t != self.frames - 1:
             raise ValueError("only a transient last frame rolls back")
         row = self.frame_pages.pop(t)
@@ -296,7 +296,7 @@ class GcaOracle:
     numpy); they are widened exactly. `slot_of(g)` names the distinct input frame that frame g
     reuses (identity by default), so long streams keep a bounded set of raw frames in memory.
     Cache frame (slot) t holds video frame gidx[t]: t itself unless `append` was given another
-    global index (keyframe streams, R7); its RoPE time position and its inputs are those of
+    global index (keyframe streams, R11); its RoPE time position and its inputs are those of
     gidx[t].
     """
 
@@ -363,7 +363,7 @@ class GcaOracle:
     # bookkeeping ----------------------------------------------------------------------
     def append(self, t, g=None, transient=False):
         """Append cache frame t holding video frame g (default t); transient: a non-keyframe
-        that will roll back (R7)."""
+        that will roll back (R11)."""
         self.book.append(t, transient)
         if g is None or g == t:
             self.gidx.pop(t, None)
@@ -423,7 +423,7 @@ class GcaOracle:
 
 
 def keyframe_stream(oracle: GcaOracle, frames: int, interval: int, on_frame=None):
-    """Streams video frames 0..frames-1 keeping every `interval`-th one (R7). After each
+    """Streams video frames 0..frames-1 keeping every `interval`-th one (R11). After each
     frame's append, `on_frame(g, slot, keyframe)` runs (the frame's attention happens there);
     a non-keyframe then rolls back. Returns the slots of the keyframes."""
     kept = []

@@ -18,7 +18,8 @@ __all__ = [
     "gca_validate_config", "gca_workspace_bytes", "gca_cache_create", "gca_append_frame",
     "gca_attend", "gca_reset", "gca_cache_destroy", "gca_check", "gca_get_state",
     "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc", "gca_append_frames",
-    "GcaCache", "config_for", "EXPORTED_SYMBOLS",
+    "gca_append_frame_ex", "gca_rollback_last_frame", "GCA_APPEND_TRANSIENT", "GcaCache",
+    "config_for", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,6 +30,7 @@ def library_path() -> str:
 
 
 GCA_OK = 0
+GCA_APPEND_TRANSIENT = 1
 STATUS = {0: "GCA_OK", -1: "GCA_ERR_INVALID_ARG", -2: "GCA_ERR_OUT_OF_PAGES",
           -3: "GCA_ERR_FRAME_ORDER", -4: "GCA_ERR_CUDA", -5: "GCA_ERR_UNSUPPORTED",
           -6: "GCA_ERR_DEVICE"}
@@ -57,7 +59,7 @@ class GcaState(ctypes.Structure):
         ("free_tail", ctypes.c_int64), ("traj_len", ctypes.c_int64),
         ("traj_pages", ctypes.c_int32), ("tokens_per_frame", ctypes.c_int32),
         ("pages_per_frame", ctypes.c_int32), ("pages_in_use", ctypes.c_int32),
-        ("device_error", ctypes.c_uint32), ("reserved", ctypes.c_int32),
+        ("device_error", ctypes.c_uint32), ("transient", ctypes.c_int32),
         ("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p),
         ("free_ring", ctypes.c_void_p), ("frame_pages", ctypes.c_void_p),
         ("traj_page_list", ctypes.c_void_p), ("slot_map", ctypes.c_void_p),
@@ -79,6 +81,7 @@ EXPORTED_SYMBOLS = (
     "gca_validate_config", "gca_workspace_bytes", "gca_cache_create", "gca_append_frame",
     "gca_attend", "gca_reset", "gca_cache_destroy", "gca_check", "gca_get_state",
     "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc", "gca_append_frames",
+    "gca_append_frame_ex", "gca_rollback_last_frame",
 )
 
 _lib = None
@@ -110,6 +113,8 @@ def lib():
         "gca_status_string": (ctypes.c_char_p, [I32]),
         "gca_attend_noalloc": (I32, [VP, I64, VP, VP, VP]),
         "gca_append_frames": (I32, [P(VP), I32, P(I64), P(VP), P(VP), P(VP), P(VP), VP]),
+        "gca_append_frame_ex": (I32, [VP, I64, I64, ctypes.c_uint32, VP, VP, VP, VP, VP]),
+        "gca_rollback_last_frame": (I32, [VP, I64, VP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -147,6 +152,16 @@ def gca_cache_create(cfg: GcaConfig, workspace_ptr: int, workspace_bytes: int,
 def gca_append_frame(handle, frame_idx, q_ptr, k_ptr, v_ptr, q_rot_ptr, stream) -> None:
     _ok(lib().gca_append_frame(handle, frame_idx, q_ptr, k_ptr, v_ptr, q_rot_ptr, stream),
         "gca_append_frame")
+
+
+def gca_append_frame_ex(handle, frame_idx, rope_frame, flags, q_ptr, k_ptr, v_ptr, q_rot_ptr,
+                        stream) -> None:
+    _ok(lib().gca_append_frame_ex(handle, frame_idx, rope_frame, flags, q_ptr, k_ptr, v_ptr,
+                                  q_rot_ptr, stream), "gca_append_frame_ex")
+
+
+def gca_rollback_last_frame(handle, frame_idx, stream=None) -> None:
+    _ok(lib().gca_rollback_last_frame(handle, frame_idx, stream), "gca_rollback_last_frame")
 
 
 def gca_attend(handle, frame_idx, q_rot_ptr, out_ptr, stream) -> None:
@@ -244,9 +259,20 @@ class GcaCache:
             pass
 
     # ------------------------------------------------------------------ hot path
-    def append_frame(self, t, q, k, v, q_rot, stream=None):
-        gca_append_frame(self.handle, t, q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                         q_rot.data_ptr(), _stream_handle(stream))
+    def append_frame(self, t, q, k, v, q_rot, stream=None, rope_frame=None, transient=False):
+        """Appends cache frame t; rope_frame (default t) is its RoPE time position; transient:
+        a non-keyframe that is rolled back after its attention."""
+        if rope_frame is None and not transient:
+            gca_append_frame(self.handle, t, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                             q_rot.data_ptr(), _stream_handle(stream))
+        else:
+            gca_append_frame_ex(self.handle, t, t if rope_frame is None else rope_frame,
+                                GCA_APPEND_TRANSIENT if transient else 0, q.data_ptr(),
+                                k.data_ptr(), v.data_ptr(), q_rot.data_ptr(),
+                                _stream_handle(stream))
+
+    def rollback(self, t):
+        gca_rollback_last_frame(self.handle, t)
 
     def attend(self, t, q_rot, out, stream=None):
         gca_attend(self.handle, t, q_rot.data_ptr(), out.data_ptr(), _stream_handle(stream))

@@ -146,8 +146,10 @@ bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams
     w0 = 0;
     nwf = 0;
   } else {
+    // A pending transient frame was appended without evicting: the window still holds the
+    // frame that a kept append would have evicted.
     na_frames = cf.anchor_frames;
-    w0 = std::max<int64_t>(cf.anchor_frames, t - cf.window_frames + 1);
+    w0 = std::max<int64_t>(cf.anchor_frames, t - cf.window_frames + (c->transient ? 0 : 1));
     nwf = t - w0 + 1;
   }
   std::memset(p, 0, sizeof(*p));
@@ -324,16 +326,20 @@ gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t w
 namespace {
 
 // Checks one append and fills its launch parameters from the host mirror; changes nothing.
-gca_status prepare_append(gca_cache* c, int64_t t, const void* q, const void* k,
-                          const void* v, void* q_rot_out, AppendParams* out) {
+gca_status prepare_append(gca_cache* c, int64_t t, int64_t rope_frame, uint32_t flags,
+                          const void* q, const void* k, const void* v, void* q_rot_out,
+                          AppendParams* out) {
   if (!c || !q || !k || !v || !q_rot_out) return GCA_ERR_INVALID_ARG;
-  if (t != c->frames) return GCA_ERR_FRAME_ORDER;
+  if ((flags & ~(uint32_t)GCA_APPEND_TRANSIENT) != 0u) return GCA_ERR_INVALID_ARG;
+  if (t != c->frames || c->transient) return GCA_ERR_FRAME_ORDER;
   if (t >= c->cfg.max_frames) return GCA_ERR_INVALID_ARG;
+  if (rope_frame < 0 || rope_frame >= c->cfg.max_frames) return GCA_ERR_INVALID_ARG;
   if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;
   const Layout& L = c->lay;
   const gca_config& cf = c->cfg;
+  const bool transient = (flags & GCA_APPEND_TRANSIENT) != 0u;
   const int64_t e = t - cf.window_frames;
-  const bool evict = e >= cf.anchor_frames;
+  const bool evict = !transient && e >= cf.anchor_frames;
   const int K = evict ? c->n_kept : 0;
   const int64_t pages_before = (c->traj_len + kPageSize - 1) / kPageSize;
   const int64_t pages_after = (c->traj_len + K + kPageSize - 1) / kPageSize;
@@ -358,6 +364,7 @@ gca_status prepare_append(gca_cache* c, int64_t t, const void* q, const void* k,
   p.rope_tok = at<float2>(c, L.rope_tok);
   p.err = at<uint32_t>(c, L.err);
   p.t = t;
+  p.rope_frame = rope_frame;
   p.traj_len = c->traj_len;
   p.head_pos = (int32_t)(c->free_head % cf.num_pages);
   p.tail_pos = (int32_t)(c->free_tail % cf.num_pages);
@@ -389,23 +396,41 @@ gca_status prepare_append(gca_cache* c, int64_t t, const void* q, const void* k,
 }
 
 // Advances the host mirror past an enqueued append.
-void commit_append(gca_cache* c, const AppendParams& p) {
+void commit_append(gca_cache* c, const AppendParams& p, bool transient) {
   c->free_head += c->lay.ppf + p.n_pop_traj;
   if (p.evict_frame >= 0) c->free_tail += c->lay.ppf;
   c->traj_len += p.K;
   c->traj_pages += p.n_pop_traj;
   c->frames += 1;
+  c->transient = transient;
 }
 
 }  // namespace
 
-gca_status gca_append_frame(gca_cache* c, int64_t t, const void* q, const void* k,
-                            const void* v, void* q_rot_out, void* stream) {
+gca_status gca_append_frame_ex(gca_cache* c, int64_t t, int64_t rope_frame, uint32_t flags,
+                               const void* q, const void* k, const void* v, void* q_rot_out,
+                               void* stream) {
   AppendParams p;
-  const gca_status st = prepare_append(c, t, q, k, v, q_rot_out, &p);
+  const gca_status st = prepare_append(c, t, rope_frame, flags, q, k, v, q_rot_out, &p);
   if (st != GCA_OK) return st;
   if (launch_append(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GCA_ERR_CUDA;
-  commit_append(c, p);
+  commit_append(c, p, (flags & GCA_APPEND_TRANSIENT) != 0u);
+  return GCA_OK;
+}
+
+gca_status gca_append_frame(gca_cache* c, int64_t t, const void* q, const void* k,
+                            const void* v, void* q_rot_out, void* stream) {
+  return gca_append_frame_ex(c, t, t, 0u, q, k, v, q_rot_out, stream);
+}
+
+gca_status gca_rollback_last_frame(gca_cache* c, int64_t t, void* /*stream*/) {
+  if (!c) return GCA_ERR_INVALID_ARG;
+  if (!c->transient || c->frames == 0 || t != c->frames - 1) return GCA_ERR_FRAME_ORDER;
+  // A transient append popped exactly ppf pages from the head and pushed none; moving the
+  // head back returns them in reverse order (the ring still holds their ids).
+  c->free_head -= c->lay.ppf;
+  c->frames -= 1;
+  c->transient = false;
   return GCA_OK;
 }
 
@@ -427,14 +452,15 @@ gca_status gca_append_frames(gca_cache* const* caches, int32_t n, const int64_t*
         c->cfg.num_heads != caches[0]->cfg.num_heads) {
       return GCA_ERR_INVALID_ARG;
     }
-    const gca_status st = prepare_append(c, frame_idx[i], q[i], k[i], v[i], q_rot_out[i], &b.p[i]);
+    const gca_status st =
+        prepare_append(c, frame_idx[i], frame_idx[i], 0u, q[i], k[i], v[i], q_rot_out[i], &b.p[i]);
     if (st != GCA_OK) return st;
     b.max_blocks = std::max(b.max_blocks, b.p[i].n_blocks);
   }
   if (launch_append_batch(b, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     return GCA_ERR_CUDA;
   }
-  for (int32_t i = 0; i < n; ++i) commit_append(caches[i], b.p[i]);
+  for (int32_t i = 0; i < n; ++i) commit_append(caches[i], b.p[i], false);
   return GCA_OK;
 }
 
@@ -481,6 +507,7 @@ gca_status gca_reset(gca_cache* c, void* stream) {
   c->free_tail = c->cfg.num_pages;
   c->traj_len = 0;
   c->traj_pages = 0;
+  c->transient = false;
   c->dev_err = 0;
   std::memset(&c->last, 0, sizeof(c->last));
   return GCA_OK;
@@ -516,6 +543,7 @@ gca_status gca_get_state(const gca_cache* c, gca_state* s) {
   s->pages_per_frame = L.ppf;
   s->pages_in_use = (int32_t)(c->cfg.num_pages - (c->free_tail - c->free_head));
   s->device_error = c->dev_err;
+  s->transient = c->transient ? 1 : 0;
   s->k_pool = c->ws + L.k_pool;
   s->v_pool = c->ws + L.v_pool;
   s->free_ring = reinterpret_cast<int32_t*>(c->ws + L.free_ring);

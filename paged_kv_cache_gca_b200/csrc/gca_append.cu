@@ -156,7 +156,8 @@ __device__ __forceinline__ void append_block(const AppendParams& p, const int bx
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const int j = 4 * c + w;  // pair index within the head
-      cs[w] = j < p.nt ? p.rope_t[p.t * p.nt + j] : p.rope_tok[(int64_t)i * p.nyx + (j - p.nt)];
+      cs[w] = j < p.nt ? p.rope_t[p.rope_frame * p.nt + j]
+                     : p.rope_tok[(int64_t)i * p.nyx + (j - p.nt)];
     }
     uint4 qr, kr;
     qr.x = rotate_word(qv.x, cs[0]);

@@ -84,7 +84,8 @@ struct AppendParams {
   const float2* rope_t;
   const float2* rope_tok;
   uint32_t* err;
-  int64_t t;
+  int64_t t;           // cache frame (page-table row)
+  int64_t rope_frame;  // RoPE time position (global frame index)
   int64_t traj_len;
   int32_t head_pos;           // free_head mod num_pages: ring position of the first pop
   int32_t tail_pos;           // free_tail mod num_pages: ring position of the first push
@@ -180,6 +181,7 @@ struct gca_cache {
   int64_t free_tail;
   int64_t traj_len;
   int32_t traj_pages;
+  bool transient;  // the last append was a non-keyframe awaiting rollback
   int32_t n_kept;
   int32_t kept[gca::kMaxKeep];
   uint32_t dev_err;

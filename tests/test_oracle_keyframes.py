@@ -1,4 +1,4 @@
-"""Pins of the oracle's keyframe-only caching (reading R7): transient append, rollback and
+"""Pins of the oracle's keyframe-only caching (reading R11): transient append, rollback and
 the keyframe stream driver, each against something other than the code under test.
 
 - a dense brute force that restates the visibility rule in video-frame terms (keys built from
@@ -95,9 +95,12 @@ def test_rollback_restores_the_allocator_exactly():
     for s in range(25):
         for _ in range(rng.randrange(4)):  # non-keyframes between keyframes
             head = list(mixed.alloc.free)[:mixed.ppf]
+            traj_before = list(mixed.traj_tokens)
+            live_before = sorted(mixed.frame_pages)
             mixed.append(s, transient=True)
             assert mixed.frame_pages[s] == head  # the pages the next keyframe will take
-            assert s - mixed.W not in mixed.traj_tokens  # nothing evicted
+            assert mixed.traj_tokens == traj_before  # nothing evicted ...
+            assert sorted(mixed.frame_pages) == live_before + [s]  # ... every frame still live
             mixed.rollback(s)
         plain.append(s)
         mixed.append(s)
