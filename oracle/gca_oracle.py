@@ -49,6 +49,11 @@ Readings where the pages are silent (each is listed in the design notes):
      frame at slot s sees the anchors, window slots max(A, s-W)..s (up to W+1 frames, itself
      included) and the kept tokens of slots A..s-W-1. The RoPE time position of a slot is the
      global index g of the video frame it holds [GCT, 3D RoPE]; without keyframes g = slot.
+  R12 scale-frame prefill [GCT, Streaming Inference API step 2 and the FAQ on scale frames]:
+     the first n scale frames (n <= A: they become the anchor pool) are processed jointly
+     with bidirectional attention: after their appends, the queries of all n frames (frame
+     by frame, n*T rows) attend over every token of frames 0..n-1, with no mask across them.
+     Streaming then continues causally (R3).
 """
 from __future__ import annotations
 
@@ -409,6 +414,26 @@ class GcaOracle:
             v[sel] = vr[tokens[sel], h, :]
         k = rotate_pairs(k[:, None, :], angles)[:, 0, :]
         return k, v
+
+    def attend_prefill(self, n, rows=None):
+        """fp64 output [len(rows), H, D] of the joint (bidirectional) attention of scale frames
+        0..n-1 (R12); rows index the n*T concatenated query rows (frame-major)."""
+        if not (1 <= n <= max(self.A, 1)) or self.book.frames != n:
+            raise ValueError("prefill needs exactly the first n <= A frames appended")
+        r = np.arange(n * self.T) if rows is None else np.asarray(rows)
+        frame_of, tok_of = r // self.T, r % self.T
+        qr = np.empty((len(r), self.H, self.D), dtype=np.float64)
+        for f in np.unique(frame_of):
+            sel = np.nonzero(frame_of == f)[0]
+            qr[sel] = self.q_rot(int(f), tok_of[sel])
+        frames = np.repeat(np.arange(n, dtype=np.int64), self.T)
+        tokens = np.tile(np.arange(self.T, dtype=np.int64), n)
+        angles = rope_angles(self.positions(frames, tokens), self.D, self.base)
+        out = np.empty_like(qr)
+        for h in range(self.H):
+            k, v = self.gather_head(n - 1, h, frames, tokens, angles)
+            out[:, h, :] = softmax_attention(qr[:, h, :], k, v)
+        return out
 
     def attend(self, t, rows=None):
         """fp64 attention output [len(rows), H, D] of frame t's query rows."""

@@ -1,5 +1,7 @@
-"""Pins of the oracle's keyframe-only caching (reading R11): transient append, rollback and
-the keyframe stream driver, each against something other than the code under test.
+"""Pins of the oracle's streaming modes beyond the plain stream, each against something other
+than the code under test.
+
+Keyframe-only caching (reading R11): transient append, rollback and the keyframe stream driver.
 
 - a dense brute force that restates the visibility rule in video-frame terms (keys built from
   the raw inputs, an explicit mask, torch's scaled_dot_product_attention in fp64);
@@ -9,6 +11,10 @@ the keyframe stream driver, each against something other than the code under tes
   exactly what a normal frame of a cache with one more window frame sees;
 - interval 1, which is the plain stream;
 - the closed form of the transient frame's visible-key count, and brute force over the book.
+
+Scale-frame prefill (reading R12): a dense unmasked SDPA brute force over the concatenated
+frames; the last scale frame's rows equal its causal rows (same key set); an earlier frame's
+rows change with a later frame's keys (bidirectional), its causal rows do not.
 """
 import random
 
@@ -171,3 +177,54 @@ def test_transient_visible_count_closed_form(A, W):
         anchor, window, evicted = orc.pool_frames(s, A, W, transient=True)
         assert sorted(book.frame_pages) == anchor + window
         assert sorted({e for e, _ in book.traj_tokens}) == evicted
+
+
+# ---------------------------------------------------------------- scale-frame prefill (R12)
+
+def dense_prefill(o, n):
+    """Brute force: the n*T queries of frames 0..n-1 against every token of those frames,
+    no mask, torch's scaled_dot_product_attention in fp64 (keys from the raw inputs)."""
+    q = torch.from_numpy(np.concatenate([_rotated(o, f, 0) for f in range(n)]))
+    k = torch.from_numpy(np.concatenate([_rotated(o, f, 1) for f in range(n)]))
+    v = torch.from_numpy(np.concatenate([o.source(f)[2].float().numpy() for f in range(n)])
+                         .astype(np.float64))
+    out = torch.nn.functional.scaled_dot_product_attention(
+        q.permute(1, 0, 2), k.permute(1, 0, 2), v.permute(1, 0, 2))
+    return out.permute(1, 0, 2).numpy()
+
+
+@pytest.mark.parametrize("n,A", [(1, 1), (3, 4), (4, 4), (2, 2)])
+def test_prefill_matches_dense_sdpa(n, A):
+    o = make_oracle(A=A, W=2, K=3)
+    for t in range(n):
+        o.append(t)
+    np.testing.assert_allclose(o.attend_prefill(n), dense_prefill(o, n), rtol=0, atol=1e-12)
+    rows = np.array([0, o.T - 1, o.T, n * o.T - 1])
+    rows = rows[rows < n * o.T]
+    np.testing.assert_allclose(o.attend_prefill(n, rows), o.attend_prefill(n)[rows], rtol=0,
+                               atol=1e-13)  # BLAS blocks by shape: equal to rounding
+
+
+def test_prefill_last_frame_rows_are_the_causal_rows():
+    o = make_oracle(A=4, W=2, K=3)
+    for t in range(4):
+        o.append(t)
+    last = o.attend_prefill(4)[3 * o.T:]
+    np.testing.assert_allclose(last, o.attend(3), rtol=0, atol=1e-13)
+
+
+def test_prefill_is_bidirectional():
+    # changing a later scale frame changes an earlier frame's rows (it would not, causally)
+    base = make_oracle(A=3, W=2, K=3)
+    other = make_oracle(A=3, W=2, K=3)
+    k2 = torch.randn(other.T, other.H, other.D).to(torch.bfloat16)
+    src = other.source
+    other.source = lambda g: (src(g)[0], k2, src(g)[2]) if g == 2 else src(g)
+    for o in (base, other):
+        for t in range(3):
+            o.append(t)
+    a, b = base.attend_prefill(3), other.attend_prefill(3)
+    assert np.abs(a[:base.T] - b[:base.T]).max() > 1e-6  # frame 0 sees frame 2's keys
+    np.testing.assert_array_equal(base.attend(0), other.attend(0))  # causally it does not
+    with pytest.raises(ValueError):
+        base.attend_prefill(2)  # three frames are appended
