@@ -231,6 +231,8 @@ def run_ours(args, rank, world, device):
     # ---- end-to-end through the public API with host buffers (pinned), copies timed
     e2e = run_e2e(args, w, cache, ring_host, device, stream, world)
     batched = run_batched_append(ring, device, stream) if world == 1 else None
+    prefill = run_prefill(ring, device, stream) if world == 1 else None
+    keyframes = run_keyframe_stream(ring, device, stream) if world == 1 else None
 
     res = {
         "elapsed_ms": elapsed_ms,
@@ -243,9 +245,97 @@ def run_ours(args, rank, world, device):
         "e2e": e2e,
         "frames": nframes,
         "batched_append": batched,
+        "prefill": prefill,
+        "keyframes": keyframes,
     }
     cache.close()
     return w, res
+
+
+def run_prefill(ring, device, stream, warm=3, timed=10):
+    """Joint bidirectional attention of the 8 scale frames (gca_attend_prefill): 8*T = 8032
+    queries over 8032 keys per head, 264 GFLOP. Frames from the device ring."""
+    import paged_kv_cache_gca_b200 as gca
+
+    w = gi.workload("scale8")
+    n = w.anchor_frames
+    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    with torch.cuda.stream(stream):
+        cache = gca.GcaCache(gca.config_for(w), initial_free=gi.initial_free_list(w),
+                             stream=stream)
+    q_all = torch.empty((n * T, H, D), dtype=torch.bfloat16, device=device)
+    out = torch.empty_like(q_all)
+    with torch.cuda.stream(stream):
+        for t in range(n):
+            q, k, v = ring[t % ring.shape[0]]
+            cache.append_frame(t, q, k, v, q_all[t * T:(t + 1) * T], stream=stream)
+        for _ in range(warm):
+            cache.attend_prefill(n, q_all, out, stream=stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(timed):
+            cache.attend_prefill(n, q_all, out, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    assert cache.check() == 0, "device error in the prefill"
+    ms = e0.elapsed_time(e1) / timed
+    flops = 4.0 * H * D * (n * T) * (n * T)
+    inf = cache.attend_info()
+    cache.close()
+    return {"workload": f"{w.name}: joint attention of {n} scale frames ({n * T} queries x "
+                        f"{n * T} keys per head, no mask across frames)",
+            "us": ms * 1e3, "flops": flops, "tflops": flops / (ms / 1e3) / 1e12,
+            "grid": inf.grid, "launches": inf.launches, "timed_calls": timed}
+
+
+def run_keyframe_stream(ring, device, stream, interval=5):
+    """The 320-frame stream with keyframe-only caching: every 5th video frame is kept, the
+    others append transiently, attend and roll back (one untimed pass, one timed pass)."""
+    import paged_kv_cache_gca_b200 as gca
+
+    w = gi.workload(WORKLOAD)
+    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    with torch.cuda.stream(stream):
+        cache = gca.GcaCache(gca.config_for(w), initial_free=gi.initial_free_list(w),
+                             stream=stream)
+    q_rot = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
+    out = torch.empty_like(q_rot)
+    flops = [0.0]
+
+    def one_pass(count):
+        cache.reset(stream=stream)
+        slot = 0
+        for g in range(w.frames):
+            q, k, v = ring[g % w.ring]
+            key = g % interval == 0
+            cache.append_frame(slot, q, k, v, q_rot, stream=stream, rope_frame=g,
+                               transient=not key)
+            cache.attend(slot, q_rot, out, stream=stream)
+            if count:
+                flops[0] += 4.0 * H * D * T * cache.attend_info().visible_keys
+            if key:
+                slot += 1
+            else:
+                cache.rollback(slot)
+
+    with torch.cuda.stream(stream):
+        one_pass(False)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        one_pass(True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    assert cache.check() == 0, "device error in the keyframe stream"
+    ms = e0.elapsed_time(e1)
+    cache.close()
+    return {"workload": f"{w.name} with keyframe interval {interval}: {w.frames} video frames, "
+                        f"{-(-w.frames // interval)} kept",
+            "frames_per_s": w.frames / (ms / 1e3), "ms_per_stream": ms,
+            "tflops_incl_append": flops[0] / (ms / 1e3) / 1e12}
 
 
 def run_batched_append(ring, device, stream, warm=16, timed=32):
@@ -550,6 +640,16 @@ def main():
             "frac": b["gbs"] / pk["hbm_gbs"], "peak_kind": pk_kind,
             **{k: v for k, v in b.items() if k != "gbs"},
         }
+    if r["prefill"] is not None:
+        pf = r["prefill"]
+        line["prefill_roofline"] = {
+            "kernel": "gca_attend_prefill (tcgen05 attention, 8032 queries, + combine)",
+            "bound": "tensor", "achieved": pf["tflops"], "peak": peak_t, "unit": "TFLOP/s",
+            "frac": pf["tflops"] / peak_t, "peak_kind": f"bf16 sustained, {pk_kind}",
+            **{k: v for k, v in pf.items() if k != "tflops"},
+        }
+    if r["keyframes"] is not None:
+        line["keyframe_stream"] = r["keyframes"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, d = oracle_frames_per_s(w, [w.frames // 2, w.frames - 1])
         line["cpu_baseline"] = {

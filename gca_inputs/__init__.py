@@ -76,7 +76,9 @@ def rope_base_for_layer(w: Workload, layer: int) -> float:
     return w.rope_base * (2.0 ** (layer / 4.0))
 
 
-# Five workloads. num_pages leaves a little headroom above the peak a stream needs.
+# The five stream workloads, then the scale-frame workload (8 scale frames processed jointly,
+# which become the anchors, then a causal window of 16). num_pages leaves a little headroom
+# above the peak a stream needs.
 WORKLOADS = {
     "tiny": Workload(
         name="tiny", num_heads=2, head_dim=64, page_size=16, grid_h=8, grid_w=8,
@@ -103,6 +105,11 @@ WORKLOADS = {
         num_special=5, anchor_frames=0, window_frames=12, keep_tokens=0, frames=500,
         seed=4, value_scale=0.125, permuted_free_list=False, ring=64, num_pages=832,
         max_frames=500, num_layers=24, num_streams=4, rope_base_varies_by_layer=True),
+    "scale8": Workload(
+        name="scale8", num_heads=16, head_dim=64, page_size=16, grid_h=37, grid_w=27,
+        num_special=5, anchor_frames=8, window_frames=16, keep_tokens=12, frames=48,
+        seed=5, value_scale=0.125, permuted_free_list=True, ring=64, num_pages=1650,
+        max_frames=48),
 }
 
 

@@ -191,6 +191,18 @@ gca_status gca_append_frames(gca_cache* const* caches, int32_t n, const int64_t*
 gca_status gca_attend(gca_cache* cache, int64_t frame_idx, const void* q_rot, void* out,
                       void* stream);
 
+/* Joint attention of the first n frames (the scale frames), bidirectional: after exactly n
+ * appends (n <= anchor_frames, so all n frames are anchors), the n*T queries of frames 0..n-1
+ * attend over every token of those frames, with no mask across frames (pages: the scale frames
+ * are processed jointly with bidirectional attention, then streaming switches to causal;
+ * Streaming Inference API, FAQ on scale frames). q_rot: device bf16 [n*T][H][D], the q_rot
+ * outputs of the n appends back to back (frame-major); out: device bf16 [n*T][H][D]. One
+ * attention launch (+ one combine launch when split). GCA_ERR_INVALID_ARG unless
+ * 1 <= n <= anchor_frames; GCA_ERR_FRAME_ORDER unless exactly n frames are appended (and no
+ * transient frame is pending). */
+gca_status gca_attend_prefill(gca_cache* cache, int32_t n, const void* q_rot, void* out,
+                              void* stream);
+
 /* The same attention as gca_attend, for callers that may not allocate device memory while
  * they run: a process that budgets all GPU memory when it starts and treats any later
  * cudaMalloc as a failure, a plugin whose host application owns the device allocator, or a

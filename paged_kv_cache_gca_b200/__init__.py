@@ -18,8 +18,8 @@ __all__ = [
     "gca_validate_config", "gca_workspace_bytes", "gca_cache_create", "gca_append_frame",
     "gca_attend", "gca_reset", "gca_cache_destroy", "gca_check", "gca_get_state",
     "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc", "gca_append_frames",
-    "gca_append_frame_ex", "gca_rollback_last_frame", "GCA_APPEND_TRANSIENT", "GcaCache",
-    "config_for", "EXPORTED_SYMBOLS",
+    "gca_append_frame_ex", "gca_rollback_last_frame", "gca_attend_prefill",
+    "GCA_APPEND_TRANSIENT", "GcaCache", "config_for", "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -81,7 +81,7 @@ EXPORTED_SYMBOLS = (
     "gca_validate_config", "gca_workspace_bytes", "gca_cache_create", "gca_append_frame",
     "gca_attend", "gca_reset", "gca_cache_destroy", "gca_check", "gca_get_state",
     "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc", "gca_append_frames",
-    "gca_append_frame_ex", "gca_rollback_last_frame",
+    "gca_append_frame_ex", "gca_rollback_last_frame", "gca_attend_prefill",
 )
 
 _lib = None
@@ -115,6 +115,7 @@ def lib():
         "gca_append_frames": (I32, [P(VP), I32, P(I64), P(VP), P(VP), P(VP), P(VP), VP]),
         "gca_append_frame_ex": (I32, [VP, I64, I64, ctypes.c_uint32, VP, VP, VP, VP, VP]),
         "gca_rollback_last_frame": (I32, [VP, I64, VP]),
+        "gca_attend_prefill": (I32, [VP, I32, VP, VP, VP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -162,6 +163,10 @@ def gca_append_frame_ex(handle, frame_idx, rope_frame, flags, q_ptr, k_ptr, v_pt
 
 def gca_rollback_last_frame(handle, frame_idx, stream=None) -> None:
     _ok(lib().gca_rollback_last_frame(handle, frame_idx, stream), "gca_rollback_last_frame")
+
+
+def gca_attend_prefill(handle, n, q_rot_ptr, out_ptr, stream) -> None:
+    _ok(lib().gca_attend_prefill(handle, n, q_rot_ptr, out_ptr, stream), "gca_attend_prefill")
 
 
 def gca_attend(handle, frame_idx, q_rot_ptr, out_ptr, stream) -> None:
@@ -276,6 +281,11 @@ class GcaCache:
 
     def attend(self, t, q_rot, out, stream=None):
         gca_attend(self.handle, t, q_rot.data_ptr(), out.data_ptr(), _stream_handle(stream))
+
+    def attend_prefill(self, n, q_rot, out, stream=None):
+        """Joint bidirectional attention of the first n frames (q_rot, out: [n*T, H, D])."""
+        gca_attend_prefill(self.handle, n, q_rot.data_ptr(), out.data_ptr(),
+                           _stream_handle(stream))
 
     def reset(self, stream=None):
         gca_reset(self.handle, _stream_handle(stream))

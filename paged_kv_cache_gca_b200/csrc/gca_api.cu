@@ -109,7 +109,10 @@ bool compute_layout(const gca_config& c, Layout* L) {
                                                    c.window_frames);
   const int64_t traj_tokens = evicted * c.keep_tokens;
   L->traj_cap_pages = (traj_tokens + kPageSize - 1) / kPageSize + 1;
-  L->part_slots = kMaxGrid + c.num_heads * L->n_qt;
+  // partial records: a launch needs 2 * (grid + units2) <= kMaxGrid + H * n_qt; the largest
+  // query set is the joint prefill of the A scale frames (A * T rows)
+  const int64_t max_q_rows = std::max<int64_t>(T, (int64_t)c.anchor_frames * T);
+  L->part_slots = kMaxGrid + c.num_heads * (int32_t)((max_q_rows + kTileQ - 1) / kTileQ);
   const size_t page_bytes = (size_t)c.num_heads * kPageSize * c.head_dim * 2;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -137,7 +140,7 @@ bool compute_layout(const gca_config& c, Layout* L) {
 }
 
 bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams* p,
-                    bool* split, int64_t* visible_keys) {
+                    bool* split, int64_t* visible_keys, int64_t q_rows) {
   const Layout& L = c->lay;
   const gca_config& cf = c->cfg;
   int64_t na_frames, w0, nwf;
@@ -156,7 +159,9 @@ bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams
   p->frame_pages = reinterpret_cast<const int32_t*>(c->ws + L.frame_pages);
   p->traj_pages = reinterpret_cast<const int32_t*>(c->ws + L.traj_pages);
   p->err = reinterpret_cast<uint32_t*>(c->ws + L.err);
-  p->T = L.T;
+  if (q_rows <= 0) q_rows = L.T;
+  const int32_t n_qt = (int32_t)((q_rows + kTileQ - 1) / kTileQ);
+  p->T = (int32_t)q_rows;
   p->H = cf.num_heads;
   p->ppf = L.ppf;
   p->last_len = L.last_len;
@@ -169,9 +174,9 @@ bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams
       c->traj_pages > 0 ? (int32_t)(c->traj_len - (int64_t)(c->traj_pages - 1) * kPageSize) : 0;
   p->n_lp = p->na_pages + p->nw_pages + p->n_traj_pages;
   p->n_tiles = (p->n_lp + kPagesPerTile - 1) / kPagesPerTile;
-  p->n_qt = L.n_qt;
-  p->units = cf.num_heads * L.n_qt;
-  p->n_pairs = (L.n_qt + 1) / 2;
+  p->n_qt = n_qt;
+  p->units = cf.num_heads * n_qt;
+  p->n_pairs = (n_qt + 1) / 2;
   p->units2 = cf.num_heads * p->n_pairs;
   p->total = (int64_t)p->units2 * p->n_tiles;
   int64_t gmax = std::min<int64_t>(kMaxGrid, (int64_t)c->sms * c->ctas_per_sm);
@@ -464,15 +469,17 @@ gca_status gca_append_frames(gca_cache* const* caches, int32_t n, const int64_t*
   return GCA_OK;
 }
 
-gca_status gca_attend(gca_cache* c, int64_t t, const void* q_rot, void* out, void* stream) {
-  if (!c || !q_rot || !out) return GCA_ERR_INVALID_ARG;
-  if (c->frames == 0 || t != c->frames - 1) return GCA_ERR_FRAME_ORDER;
-  if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;
+namespace {
+
+// Plans and enqueues one attention of q_rows query rows (0: one frame) over the keys frame t
+// sees.
+gca_status enqueue_attention(gca_cache* c, int64_t t, int64_t q_rows, const void* q_rot,
+                             void* out, void* stream) {
   const Layout& L = c->lay;
   AttnParams p;
   bool split = false;
   int64_t nk = 0;
-  if (!plan_attention(c, t, L.part_slots, &p, &split, &nk)) return GCA_ERR_UNSUPPORTED;
+  if (!plan_attention(c, t, L.part_slots, &p, &split, &nk, q_rows)) return GCA_ERR_UNSUPPORTED;
   p.q = static_cast<const uint4*>(q_rot);
   p.out = static_cast<uint4*>(out);
   p.part_o = at<float>(c, L.part_o);
@@ -486,11 +493,30 @@ gca_status gca_attend(gca_cache* c, int64_t t, const void* q_rot, void* out, voi
   inf.visible_keys = nk;
   inf.logical_pages = p.n_lp;
   inf.kv_tiles = p.n_tiles;
-  inf.query_tiles = L.n_qt;
+  inf.query_tiles = p.n_qt;
   inf.grid = p.grid;
   inf.split = split ? 1 : 0;
   inf.launches = split ? 2 : 1;
   return GCA_OK;
+}
+
+}  // namespace
+
+gca_status gca_attend(gca_cache* c, int64_t t, const void* q_rot, void* out, void* stream) {
+  if (!c || !q_rot || !out) return GCA_ERR_INVALID_ARG;
+  if (c->frames == 0 || t != c->frames - 1) return GCA_ERR_FRAME_ORDER;
+  if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;
+  return enqueue_attention(c, t, 0, q_rot, out, stream);
+}
+
+gca_status gca_attend_prefill(gca_cache* c, int32_t n, const void* q_rot, void* out,
+                              void* stream) {
+  if (!c || !q_rot || !out) return GCA_ERR_INVALID_ARG;
+  if (n < 1 || n > c->cfg.anchor_frames) return GCA_ERR_INVALID_ARG;
+  if (c->frames != n || c->transient) return GCA_ERR_FRAME_ORDER;
+  if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;
+  // frames 0..n-1 are all anchors (n <= A), so frame n-1's key set is every token of them
+  return enqueue_attention(c, n - 1, (int64_t)n * c->lay.T, q_rot, out, stream);
 }
 
 gca_status gca_reset(gca_cache* c, void* stream) {

@@ -120,7 +120,8 @@ struct AttnParams {
   const int32_t* frame_pages;
   const int32_t* traj_pages;
   uint32_t* err;
-  int32_t T, H, ppf, last_len, num_pages;
+  int32_t T;  // query rows of the launch (T of one frame, or n * T for a joint prefill)
+  int32_t H, ppf, last_len, num_pages;
   int32_t na_pages;      // anchor pages (visible anchor frames * ppf)
   int32_t win_base;      // index into frame_pages of the first window page
   int32_t nw_pages;      // window pages
@@ -163,8 +164,9 @@ __host__ __device__ inline int64_t part_slot(int64_t cta, int64_t u2, int q) {
 // Fills the frame-dependent fields of p for gca_attend of frame t (visible page ranges, tiles,
 // work split) with at most max_slots partial-record slots; returns false if even one CTA per
 // work unit does not fit. *split: some unit spans several CTAs, so the combine kernel must run.
+// q_rows: query rows of the launch (0: one frame, T).
 bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams* p,
-                    bool* split, int64_t* visible_keys);
+                    bool* split, int64_t* visible_keys, int64_t q_rows = 0);
 
 }  // namespace gca
 

@@ -9,6 +9,11 @@ With --batch N it instead creates N caches of the workload and runs --frame + 1 
 (gca_append_frames over all N caches; frame of cache c at step t: ring slot (N t + c) mod R):
 
     python -m paged_kv_cache_gca_b200.profile_frame --workload stack24x4 --batch 16 --frame 15
+
+With --prefill it appends the workload's anchor (scale) frames and runs --repeat joint
+attentions over them (gca_attend_prefill):
+
+    python -m paged_kv_cache_gca_b200.profile_frame --workload scale8 --prefill --repeat 1
 """
 import argparse
 import os
@@ -30,9 +35,12 @@ def main():
     ap.add_argument("--frame", type=int, default=-1)
     ap.add_argument("--repeat", type=int, default=1)
     ap.add_argument("--batch", type=int, default=0)
+    ap.add_argument("--prefill", action="store_true")
     args = ap.parse_args()
     if args.batch > 0:
         return batched(args)
+    if args.prefill:
+        return prefill(args)
     w = gi.workload(args.workload)
     t_last = w.frames - 1 if args.frame < 0 else args.frame
     T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
@@ -50,6 +58,26 @@ def main():
     inf = cache.attend_info()
     print(f"{w.name} t={t_last}: Nk={inf.visible_keys} grid={inf.grid} split={inf.split} "
           f"status={status}")
+    sys.exit(0 if status == 0 else 1)
+
+
+def prefill(args):
+    w = gi.workload(args.workload)
+    n = w.anchor_frames
+    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    ring = gi.draw_ring(w, slots=n).cuda()
+    cache = gca.GcaCache(gca.config_for(w), initial_free=gi.initial_free_list(w))
+    q_all = torch.empty((n * T, H, D), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(q_all)
+    for t in range(n):
+        q, k, v = ring[t]
+        cache.append_frame(t, q, k, v, q_all[t * T:(t + 1) * T])
+    for _ in range(args.repeat):
+        cache.attend_prefill(n, q_all, out)
+    torch.cuda.synchronize()
+    status = cache.check()
+    inf = cache.attend_info()
+    print(f"{w.name} prefill of {n} frames: grid={inf.grid} split={inf.split} status={status}")
     sys.exit(0 if status == 0 else 1)
 
 

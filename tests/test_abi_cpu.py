@@ -103,6 +103,7 @@ def test_create_rejects_bad_arguments_before_touching_cuda(L):
     assert L.gca_cache_destroy(None) == 0
     assert L.gca_append_frame_ex(None, 0, 0, 0, 1, 1, 1, 1, None) == -1
     assert L.gca_rollback_last_frame(None, 0, None) == -1
+    assert L.gca_attend_prefill(None, 1, 1, 1, None) == -1
     # batched append: empty or oversized batch, null arrays, null cache
     VP, I64 = ctypes.c_void_p, ctypes.c_int64
     one = (VP * 1)(1)
