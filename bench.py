@@ -233,6 +233,8 @@ def run_ours(args, rank, world, device):
     batched = run_batched_append(ring, device, stream) if world == 1 else None
     prefill = run_prefill(ring, device, stream) if world == 1 else None
     keyframes = run_keyframe_stream(ring, device, stream) if world == 1 else None
+    camera = run_camera_head(device, stream) if world == 1 else None
+    windowed_mode = run_windowed(ring, device, stream) if world == 1 else None
 
     res = {
         "elapsed_ms": elapsed_ms,
@@ -247,6 +249,8 @@ def run_ours(args, rank, world, device):
         "batched_append": batched,
         "prefill": prefill,
         "keyframes": keyframes,
+        "camera": camera,
+        "windowed": windowed_mode,
     }
     cache.close()
     return w, res
@@ -336,6 +340,90 @@ def run_keyframe_stream(ring, device, stream, interval=5):
                         f"{-(-w.frames // interval)} kept",
             "frames_per_s": w.frames / (ms / 1e3), "ms_per_stream": ms,
             "tflops_incl_append": flops[0] / (ms / 1e3) / 1e12}
+
+
+def run_camera_head(device, stream):
+    """The causal camera head's caches (one per trunk layer, 4): one camera token per frame,
+    32 heads, window 16, K = 1. Per frame, layer by layer as a trunk runs them: append, then
+    attend (one query row per head over up to 1024 keys: the decode-like regime). One untimed
+    pass, one timed pass of the 1024-frame stream."""
+    import paged_kv_cache_gca_b200 as gca
+
+    w = gi.workload("camera4")
+    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    ring = gi.draw_ring(w).to(device)
+    with torch.cuda.stream(stream):
+        caches = [gca.GcaCache(gca.config_for(w), stream=stream) for _ in range(w.num_layers)]
+    q_rot = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
+    out = torch.empty_like(q_rot)
+
+    def one_pass():
+        for c in caches:
+            c.reset(stream=stream)
+        for t in range(w.frames):
+            q, k, v = ring[t % w.ring]
+            for c in caches:
+                c.append_frame(t, q, k, v, q_rot, stream=stream)
+                c.attend(t, q_rot, out, stream=stream)
+
+    with torch.cuda.stream(stream):
+        one_pass()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        one_pass()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    assert all(c.check() == 0 for c in caches), "device error in the camera head caches"
+    ms = e0.elapsed_time(e1)
+    for c in caches:
+        c.close()
+    return {"workload": f"{w.name}: causal camera head caches, {w.num_layers} trunk layers, 1 "
+                        f"camera token x {H} heads x {D} per frame, anchor {w.anchor_frames}, "
+                        f"window {w.window_frames}, K {w.keep_tokens}, {w.frames} frames",
+            "frames_per_s": w.frames / (ms / 1e3),
+            "us_per_layer_frame": ms * 1e3 / (w.frames * w.num_layers)}
+
+
+def run_windowed(ring, device, stream, total=1000, window=128, overlap=8):
+    """Windowed mode (--mode windowed --window_size 128 --overlap_keyframes 8) over a
+    1000-frame video on the w16_320 layer: the cache restarts every 120 frames and re-streams
+    the 8 overlap frames. One untimed pass, one timed pass."""
+    import paged_kv_cache_gca_b200 as gca
+    from paged_kv_cache_gca_b200 import windowed
+
+    w = gi.workload(WORKLOAD).replace(max_frames=window)
+    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    with torch.cuda.stream(stream):
+        cache = gca.GcaCache(gca.config_for(w), initial_free=gi.initial_free_list(w),
+                             stream=stream)
+    drv = windowed.WindowedStream(cache, window, overlap)
+    q_rot = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
+    out = torch.empty_like(q_rot)
+    sched = list(windowed.windowed_schedule(total, window, overlap))
+
+    def one_pass():
+        for _, g, loc in sched:
+            q, k, v = ring[g % ring.shape[0]]
+            drv.step(loc, q, k, v, q_rot, out, stream=stream)
+
+    with torch.cuda.stream(stream):
+        one_pass()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        one_pass()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    assert cache.check() == 0, "device error in the windowed stream"
+    ms = e0.elapsed_time(e1)
+    cache.close()
+    return {"workload": f"{w.name} layer, windowed mode: {total} video frames, window {window}, "
+                        f"overlap {overlap} ({sched[-1][0] + 1} windows, {len(sched)} frames "
+                        "streamed)",
+            "video_frames_per_s": total / (ms / 1e3), "ms": ms}
 
 
 def run_batched_append(ring, device, stream, warm=16, timed=32):
@@ -650,6 +738,10 @@ def main():
         }
     if r["keyframes"] is not None:
         line["keyframe_stream"] = r["keyframes"]
+    if r["camera"] is not None:
+        line["camera_head"] = r["camera"]
+    if r["windowed"] is not None:
+        line["windowed_mode"] = r["windowed"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, d = oracle_frames_per_s(w, [w.frames // 2, w.frames - 1])
         line["cpu_baseline"] = {

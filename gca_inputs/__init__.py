@@ -77,8 +77,10 @@ def rope_base_for_layer(w: Workload, layer: int) -> float:
 
 
 # The five stream workloads, then the scale-frame workload (8 scale frames processed jointly,
-# which become the anchors, then a causal window of 16). num_pages leaves a little headroom
-# above the peak a stream needs.
+# which become the anchors, then a causal window of 16) and the causal camera head's cache (one
+# camera token per frame, 32 heads x 64 = its 2048-wide input, the aggregator's window policy,
+# one cache per layer of its 4-layer trunk). num_pages leaves a little headroom above the peak
+# a stream needs.
 WORKLOADS = {
     "tiny": Workload(
         name="tiny", num_heads=2, head_dim=64, page_size=16, grid_h=8, grid_w=8,
@@ -110,6 +112,11 @@ WORKLOADS = {
         num_special=5, anchor_frames=8, window_frames=16, keep_tokens=12, frames=48,
         seed=5, value_scale=0.125, permuted_free_list=True, ring=64, num_pages=1650,
         max_frames=48),
+    "camera4": Workload(
+        name="camera4", num_heads=32, head_dim=64, page_size=16, grid_h=0, grid_w=0,
+        num_special=1, anchor_frames=1, window_frames=16, keep_tokens=1, frames=1024,
+        seed=6, value_scale=0.125, permuted_free_list=False, ring=64, num_pages=96,
+        max_frames=1024, num_layers=4),
 }
 
 

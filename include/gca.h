@@ -64,9 +64,10 @@ typedef struct {
   int32_t num_heads;     /* H */
   int32_t head_dim;      /* D; 64 */
   int32_t page_size;     /* tokens per page; 16 */
-  int32_t grid_h;        /* patch rows per frame */
-  int32_t grid_w;        /* patch columns per frame */
-  int32_t num_special;   /* S: camera + register tokens; T = S + grid_h * grid_w */
+  int32_t grid_h;        /* patch rows per frame (0 with no patches) */
+  int32_t grid_w;        /* patch columns per frame (0 with no patches) */
+  int32_t num_special;   /* S: camera + register tokens; T = S + grid_h * grid_w >= 1 (a
+                          * patch-free cache, e.g. the causal camera head's: T = S = 1) */
   int32_t anchor_frames; /* A >= 0 */
   int32_t window_frames; /* W >= 1, counts the current frame */
   int32_t keep_tokens;   /* K >= 0 tokens kept per evicted frame (0: no trajectory pool) */

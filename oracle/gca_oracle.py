@@ -54,6 +54,11 @@ Readings where the pages are silent (each is listed in the design notes):
      with bidirectional attention: after their appends, the queries of all n frames (frame
      by frame, n*T rows) attend over every token of frames 0..n-1, with no mask across them.
      Streaming then continues causally (R3).
+  R14 windowed restart [LingBot-Map 10,000-frame page, "Cloning and Installing"; summary page,
+     "Main features": --mode windowed --window_size N --overlap_keyframes V]: windows of N
+     video frames, each starting N - V frames after the previous one (the last one ends at the
+     last frame); at each window start the cache restarts empty and the window's frames (the
+     previous window's last V first) stream causally with local indices g - start.
 """
 from __future__ import annotations
 
@@ -73,6 +78,7 @@ __all__ = [
     "visible_keys",
     "visible_key_count",
     "keyframe_stream",
+    "windowed_frames",
     "softmax_attention",
     "FifoPages",
     "CacheBook",
@@ -329,9 +335,13 @@ class GcaOracle:
         self._raw = {}  # slot -> (q, k, v) as float32 arrays (exact copies of bf16)
         self._pos = token_positions(0, self.S, self.gh, self.gw)
         self.gidx = {}  # cache frame -> global (video) frame index, when not the identity
+        self.rpos = {}  # cache frame -> RoPE time position, when not its global index (R14)
 
     def global_index(self, t):
         return self.gidx.get(int(t), int(t))
+
+    def rope_index(self, t):
+        return self.rpos.get(int(t), self.global_index(t))
 
     # inputs ---------------------------------------------------------------------------
     def raw32(self, t):
@@ -350,7 +360,8 @@ class GcaOracle:
         frames = np.asarray(frames, dtype=np.int64)
         tokens = np.asarray(tokens, dtype=np.int64)
         pos = self._pos[tokens].copy()
-        pos[:, 0] = [self.global_index(f) for f in frames] if self.gidx else frames
+        pos[:, 0] = ([self.rope_index(f) for f in frames] if (self.gidx or self.rpos)
+                     else frames)
         return pos
 
     def q_rot(self, t, rows=None):
@@ -366,18 +377,29 @@ class GcaOracle:
         return rotate_pairs(k, ang)
 
     # bookkeeping ----------------------------------------------------------------------
-    def append(self, t, g=None, transient=False):
-        """Append cache frame t holding video frame g (default t); transient: a non-keyframe
-        that will roll back (R11)."""
+    def append(self, t, g=None, transient=False, rope_pos=None):
+        """Append cache frame t holding video frame g (default t), rotated at time rope_pos
+        (default g); transient: a non-keyframe that will roll back (R11)."""
         self.book.append(t, transient)
         if g is None or g == t:
             self.gidx.pop(t, None)
         else:
             self.gidx[t] = int(g)
+        if rope_pos is None or rope_pos == self.global_index(t):
+            self.rpos.pop(t, None)
+        else:
+            self.rpos[t] = int(rope_pos)
 
     def rollback(self, t):
         self.book.rollback(t)
         self.gidx.pop(t, None)
+        self.rpos.pop(t, None)
+
+    def restart(self):
+        """Empty cache (reset, R14)."""
+        self.book.reset()
+        self.gidx.clear()
+        self.rpos.clear()
 
     def _transient(self, t):
         return self.book.transient and t == self.book.frames - 1
@@ -463,6 +485,19 @@ def keyframe_stream(oracle: GcaOracle, frames: int, interval: int, on_frame=None
         else:
             oracle.rollback(slot)
     return kept
+
+
+def windowed_frames(total, window, overlap):
+    """(window, video frame, local index) in processing order (R14)."""
+    out = []
+    start, w = 0, 0
+    while True:
+        end = min(start + window, total)
+        out += [(w, g, g - start) for g in range(start, end)]
+        if end >= total:
+            return out
+        start += window - overlap
+        w += 1
 
 
 def _to_f32(x):

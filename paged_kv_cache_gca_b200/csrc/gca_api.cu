@@ -16,7 +16,7 @@ namespace gca {
 
 namespace {
 
-constexpr int kMinStepsPerCta = 16;
+constexpr int kMinStepsPerCta = 4;  // small launches (decode-like caches) spread wider
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -52,15 +52,17 @@ bool encode_pool_map(CUtensorMap* map, void* base, int64_t rows) {
 
 gca_status validate(const gca_config* c) {
   if (!c) return GCA_ERR_INVALID_ARG;
-  if (c->num_heads < 1 || c->head_dim < 1 || c->page_size < 1 || c->grid_h < 1 ||
-      c->grid_w < 1 || c->num_special < 0 || c->anchor_frames < 0 || c->window_frames < 1 ||
+  if (c->num_heads < 1 || c->head_dim < 1 || c->page_size < 1 || c->grid_h < 0 ||
+      c->grid_w < 0 || c->num_special < 0 || c->anchor_frames < 0 || c->window_frames < 1 ||
       c->keep_tokens < 0 || c->max_frames < 1 || c->num_pages < 1 ||
       !(c->rope_base > 0.f) || !std::isfinite(c->rope_base)) {
     return GCA_ERR_INVALID_ARG;
   }
   const int64_t P = (int64_t)c->grid_h * c->grid_w;
   const int64_t T = c->num_special + P;
-  if (T > (1 << 24) || c->max_frames > (1 << 24)) return GCA_ERR_INVALID_ARG;
+  // T >= 1; a patch-free frame (grid 0 x 0) holds only its special tokens, e.g. the single
+  // camera token of the causal camera head's cache
+  if (T < 1 || T > (1 << 24) || c->max_frames > (1 << 24)) return GCA_ERR_INVALID_ARG;
   if (c->keep_tokens > T) return GCA_ERR_INVALID_ARG;
   if (c->keep_tokens > c->num_special && c->keep_tokens - c->num_special > P) {
     return GCA_ERR_INVALID_ARG;

@@ -228,3 +228,66 @@ def test_prefill_is_bidirectional():
     np.testing.assert_array_equal(base.attend(0), other.attend(0))  # causally it does not
     with pytest.raises(ValueError):
         base.attend_prefill(2)  # three frames are appended
+
+
+# ------------------------------------------------- patch-free cache (causal camera head, R13)
+
+def test_camera_token_cache_is_causal_attention_over_all_camera_tokens():
+    """One camera token per frame and K = 1: every evicted frame keeps its token, so frame t
+    sees the camera tokens of all frames 0..t. Brute force: torch SDPA over the rotated camera
+    tokens of frames 0..t (rotated only in time: the token sits at (t, 0, 0))."""
+    o = make_oracle(H=4, gh=0, gw=0, S=1, A=1, W=3, K=1, base=500.0)
+    for t in range(12):
+        o.append(t)
+        assert orc.visible_key_count(t, o.A, o.W, o.T, o.K) == t + 1
+        q = torch.from_numpy(_rotated(o, t, 0))
+        k = torch.from_numpy(np.concatenate([_rotated(o, f, 1) for f in range(t + 1)]))
+        v = torch.from_numpy(np.concatenate([o.source(f)[2].float().numpy()
+                                             for f in range(t + 1)]).astype(np.float64))
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q.permute(1, 0, 2), k.permute(1, 0, 2), v.permute(1, 0, 2)).permute(1, 0, 2)
+        np.testing.assert_allclose(o.attend(t), ref.numpy(), rtol=0, atol=1e-12)
+    # frame 0 sees one key: the output is its v exactly
+    o0 = make_oracle(H=4, gh=0, gw=0, S=1, A=1, W=3, K=1)
+    o0.append(0)
+    np.testing.assert_array_equal(o0.attend(0), o0.raw(0)[2])
+    assert orc.token_positions(7, 1, 0, 0).tolist() == [[7, 0, 0]]
+
+
+# ------------------------------------------------------------- windowed restart (R14)
+
+@pytest.mark.parametrize("total,N,V", [(500, 128, 8), (128, 128, 8), (129, 128, 8), (10, 4, 1),
+                                       (7, 7, 0), (1, 3, 2), (30, 5, 4)])
+def test_windowed_schedule_closed_form(total, N, V):
+    sched = orc.windowed_frames(total, N, V)
+    n_windows = 1 if total <= N else 1 + -(-(total - N) // (N - V))
+    assert sched[-1][0] == n_windows - 1
+    assert all(0 <= loc < N for _, _, loc in sched)  # RoPE positions stay in the window
+    assert sorted({g for _, g, _ in sched}) == list(range(total))  # every frame, in order
+    assert len(sched) == total + V * (n_windows - 1)  # overlap frames run twice
+    for w in range(1, n_windows):
+        prev = [g for ww, g, _ in sched if ww == w - 1]
+        cur = [g for ww, g, _ in sched if ww == w]
+        assert prev[-V:] == cur[:V] if V else not set(prev) & set(cur)
+        assert cur[0] == w * (N - V)
+
+
+def test_windowed_stream_is_a_fresh_stream_per_window():
+    """Each window's attention equals a new oracle streaming that window's frames from local
+    index 0 (frame g at local position g - start, so its RoPE time is local)."""
+    A, W, K, N, V = 1, 2, 3, 5, 2
+    o = make_oracle(A=A, W=W, K=K)
+    outs = {}
+    for w, g, loc in orc.windowed_frames(12, N, V):
+        if loc == 0:
+            o.restart()
+        o.append(loc, g, rope_pos=loc)
+        outs[(w, g)] = o.attend(loc)
+    for w in range(4):
+        start = w * (N - V)
+        ref = make_oracle(A=A, W=W, K=K)
+        ref.source = (lambda s0: (lambda t: o.source(t + s0)))(start)
+        ref._raw = {}
+        for loc in range(min(N, 12 - start)):
+            ref.append(loc)
+            np.testing.assert_array_equal(outs[(w, start + loc)], ref.attend(loc))
