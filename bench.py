@@ -489,40 +489,58 @@ def run_batched_append(ring, device, stream, warm=16, timed=32):
 
 def run_e2e(args, w, cache, ring_host, device, stream, world):
     """Frames/s through the public API with inputs in pinned host memory: every frame's q, k, v
-    are copied host->device and its output device->host inside the timed region. Copies run on
-    a second stream so frame t+1's upload overlaps frame t's compute."""
+    are copied host->device and its output device->host inside the timed region. Uploads and
+    downloads run on their own streams (one copy engine each way), ordered against the compute
+    stream by events, with three rotating input and output buffers: frame t+1's upload and
+    frame t-1's download overlap frame t's compute."""
     T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    nbuf = 3
     pinned = ring_host.pin_memory()
-    out_host = torch.empty((2, T, H, D), dtype=torch.bfloat16).pin_memory()
-    inp = [torch.empty((3, T, H, D), dtype=torch.bfloat16, device=device) for _ in range(2)]
+    out_host = torch.empty((nbuf, T, H, D), dtype=torch.bfloat16).pin_memory()
+    inp = [torch.empty((3, T, H, D), dtype=torch.bfloat16, device=device) for _ in range(nbuf)]
     q_rot = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
-    out = [torch.empty((T, H, D), dtype=torch.bfloat16, device=device) for _ in range(2)]
-    copy = torch.cuda.Stream(device=device)
-    up = [torch.cuda.Event() for _ in range(2)]
-    done = [torch.cuda.Event() for _ in range(2)]
+    out = [torch.empty((T, H, D), dtype=torch.bfloat16, device=device) for _ in range(nbuf)]
+    h2d = torch.cuda.Stream(device=device)
+    d2h = torch.cuda.Stream(device=device)
+    up = [torch.cuda.Event() for _ in range(nbuf)]        # input b uploaded
+    used = [torch.cuda.Event() for _ in range(nbuf)]      # input b consumed by the append
+    ready = [torch.cuda.Event() for _ in range(nbuf)]     # output b computed
+    down = [torch.cuda.Event() for _ in range(nbuf)]      # output b downloaded
     nframes = w.frames
     steps = max(1, min(args.steps, 3))
+    started = [False] * nbuf      # input buffer b has been uploaded into before
+    downloading = [False] * nbuf  # output buffer b has a download issued (maybe in flight)
+
+    def upload(t):
+        b = t % nbuf
+        with torch.cuda.stream(h2d):
+            if started[b]:
+                h2d.wait_event(used[b])  # the append that read buffer b last has run
+            inp[b].copy_(pinned[t % w.ring], non_blocking=True)
+            up[b].record(h2d)
+        started[b] = True
 
     def step():
         cache.reset(stream=stream)
-        with torch.cuda.stream(copy):
-            inp[0].copy_(pinned[0], non_blocking=True)
-            up[0].record(copy)
+        upload(0)
+        if nframes > 1:
+            upload(1)
         for t in range(nframes):
-            b = t & 1
-            if t + 1 < nframes:
-                nb = (t + 1) & 1
-                with torch.cuda.stream(copy):
-                    if t >= 1:
-                        copy.wait_event(done[nb])  # buffer nb was last used by frame t-1
-                    inp[nb].copy_(pinned[(t + 1) % w.ring], non_blocking=True)
-                    up[nb].record(copy)
+            b = t % nbuf
+            if t + 2 < nframes:
+                upload(t + 2)
             stream.wait_event(up[b])
             cache.append_frame(t, inp[b][0], inp[b][1], inp[b][2], q_rot, stream=stream)
+            used[b].record(stream)
+            if downloading[b]:
+                stream.wait_event(down[b])  # output b's previous frame has been downloaded
             cache.attend(t, q_rot, out[b], stream=stream)
-            with torch.cuda.stream(stream):
+            ready[b].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(ready[b])
                 out_host[b].copy_(out[b], non_blocking=True)
-            done[b].record(stream)
+                down[b].record(d2h)
+            downloading[b] = True
 
     with torch.cuda.stream(stream):
         step()
@@ -535,7 +553,7 @@ def run_e2e(args, w, cache, ring_host, device, stream, world):
     e0.record(stream)
     for _ in range(steps):
         step()
-    copy.synchronize()
+    stream.wait_stream(d2h)  # the last downloads are inside the timed region
     e1.record(stream)
     torch.cuda.synchronize(device)
     ms = max_over_ranks(e0.elapsed_time(e1), world, device)

@@ -55,17 +55,8 @@
 //   GCA_TURN_EARLY the turn passes to the other warpgroup this many 32-column chunks before
 //                  this one's exponentials are done.
 //   GCA_MMA_SPIN   1: the MMA-issuing threads spin on their barriers; 0: they sleep in try_wait.
-//   GCA_SM_SPIN    1: the softmax warps spin on S, slot counts and P V completion; 0: sleep.
-//   GCA_LATE_PV    1: the softmax waits for P V of the previous tile only before it stores the
-//                  new P (after its exponentials); 0: before its turn.
 #ifndef GCA_MMA_SPIN
 #define GCA_MMA_SPIN 1
-#endif
-#ifndef GCA_SM_SPIN
-#define GCA_SM_SPIN 0
-#endif
-#ifndef GCA_LATE_PV
-#define GCA_LATE_PV 0
 #endif
 //   GCA_TURNS      1: the two softmax warpgroups take turns for the exponentials; 0: both
 //                  compute them whenever their scores are ready.
@@ -82,6 +73,21 @@
 //                  with a cubic polynomial instead of MUFU (relieves the MUFU bottleneck).
 #ifndef GCA_POLY_PAIRS
 #define GCA_POLY_PAIRS 0
+#endif
+//   GCA_F32X2      1: the scale-subtract and the row sum use packed f32x2 FMA / add (half the
+//                  instructions of the scalar forms).
+#ifndef GCA_F32X2
+#define GCA_F32X2 0
+#endif
+//   GCA_FFMA_CHUNK 1: the scale-subtract runs per 32-column chunk, just before its exponentials.
+#ifndef GCA_FFMA_CHUNK
+#define GCA_FFMA_CHUNK 0
+#endif
+//   GCA_TURN_WARP  1: the turn alternates per SM sub-partition: warp w of one warpgroup hands
+//                  it to warp w of the other (the two share that sub-partition's MUFU); 0: the
+//                  whole warpgroup hands over at once (waits for its slowest warp).
+#ifndef GCA_TURN_WARP
+#define GCA_TURN_WARP 0
 #endif
 
 #ifndef GCA_TRACE
@@ -141,7 +147,8 @@ struct __align__(8) Shared {
   uint64_t s_free[kQPerCta];
   uint64_t p_full[kQPerCta];
   uint64_t pv_done[kQPerCta];
-  uint64_t turn[kQPerCta];  // exponential turns of the two softmax warpgroups
+  uint64_t turn[kQPerCta][4];  // exponential turns of the two softmax warpgroups (per warp
+                               // when GCA_TURN_WARP, else [q][0] for the whole warpgroup)
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -263,16 +270,6 @@ __device__ __forceinline__ bool mma_wait(uint64_t* bar, uint32_t parity, Shared*
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Shared* sh,
                                           uint32_t* err, bool drain = false) {
   return __all_sync(0xffffffffu, wait_phase(bar, parity, sh, err, drain));
-}
-
-// The softmax warps' waits for S, the key-slot counts and P V completion.
-__device__ __forceinline__ bool sm_wait(uint64_t* bar, uint32_t parity, Shared* sh,
-                                        uint32_t* err) {
-#if GCA_SM_SPIN
-  return __all_sync(0xffffffffu, spin_phase(bar, parity, sh, err));
-#else
-  return warp_wait(bar, parity, sh, err);
-#endif
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -403,6 +400,24 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
 
+#if GCA_F32X2
+// x = x * c + b on a pair (packed f32x2 FMA).
+__device__ __forceinline__ void fma2_pair(float& x0, float& x1, float c, float b) {
+  asm("{\n\t.reg .b64 x, cc, bb;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 cc, {%2, %2};\n\t"
+      "mov.b64 bb, {%3, %3};\n\tfma.rn.f32x2 x, x, cc, bb;\n\tmov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "f"(c), "f"(b));
+}
+
+// (a0, a1) += (b0, b1) (packed f32x2 add).
+__device__ __forceinline__ void add2_pair(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 b, {%2, %3};\n\t"
+      "add.rn.f32x2 a, a, b;\n\tmov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+#endif
+
 __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
   __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&b);
@@ -485,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh.s_free[q], kTileQ);
       mbar_init(&sh.p_full[q], kTileQ);
       mbar_init(&sh.pv_done[q], 1);
-      mbar_init(&sh.turn[q], kTileQ);
+      for (int w = 0; w < 4; ++w) mbar_init(&sh.turn[q][w], GCA_TURN_WARP ? 1 : kTileQ);
     }
     sh.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -646,8 +661,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* q_tile = q_smem + qq * kTileBytes;
     uint32_t it = 0, turns = 0;
     bool ok = true;
+    // the turn barrier of this warp: its own sub-partition's, or the warpgroup's
+    uint64_t* const my_turn = &sh.turn[qq][GCA_TURN_WARP ? (warp & 3) : 0];
+    uint64_t* const their_turn = &sh.turn[qq ^ 1][GCA_TURN_WARP ? (warp & 3) : 0];
 #if GCA_TURNS
-    if (qq == 1) mbar_arrive(&sh.turn[0]);  // the first turn goes to query tile 0
+    if (qq == 1 && (!GCA_TURN_WARP || lane == 0)) mbar_arrive(their_turn);  // query tile 0 first
 #endif
     for (int64_t s = s_begin; s < s_end && ok;) {
       const int u2 = (int)(s / p.n_tiles);
@@ -675,9 +693,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m_run = -INFINITY;  // running row max, log2 units (scaled)
       float l_run = 0.f;        // running row sum relative to m_run
       for (int j = j0; j < j1; ++j, ++it) {
-        if (!sm_wait(&sh.s_full[qq], it & 1u, &sh, p.err)) { ok = false; break; }
+        if (!warp_wait(&sh.s_full[qq], it & 1u, &sh, p.err)) { ok = false; break; }
         if (r == 0) TRACE(16 + qq, it);
-        if (!sm_wait(&sh.lens_full[it & 3], (it >> 2) & 1u, &sh, p.err)) { ok = false; break; }
+        if (!warp_wait(&sh.lens_full[it & 3], (it >> 2) & 1u, &sh, p.err)) { ok = false; break; }
         const uint64_t lens = sh.lens[it & 3];
         if (r == 0) TRACE(6 + 5 * qq, it);
         tc_fence_after();
@@ -719,9 +737,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_new = tile_max;
           alpha = ex2(m_run - m_new);
         }
-        if (!GCA_LATE_PV && j > j0) {
+        if (j > j0) {
           // P V of the previous tile must be done before P is overwritten or O rescaled
-          if (!sm_wait(&sh.pv_done[qq], (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
+          if (!warp_wait(&sh.pv_done[qq], (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
           tc_fence_after();
         }
         if (r == 0) TRACE(7 + 5 * qq, it);
@@ -730,52 +748,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         // other warpgroup GCA_TURN_EARLY chunks before the end so that its first exponentials
         // queue behind this group's last ones.
 #if GCA_TURNS && GCA_TURN_SPIN
-        if (!__all_sync(0xffffffffu, spin_phase<(GCA_TURN_SPIN >= 2 ? GCA_TURN_SPIN : 0)>(&sh.turn[qq], turns & 1u, &sh, p.err))) {
+        if (!__all_sync(0xffffffffu, spin_phase<(GCA_TURN_SPIN >= 2 ? GCA_TURN_SPIN : 0)>(
+                                         my_turn, turns & 1u, &sh, p.err))) {
           ok = false;
           break;
         }
 #elif GCA_TURNS
-        if (!warp_wait(&sh.turn[qq], turns & 1u, &sh, p.err)) { ok = false; break; }
+        if (!warp_wait(my_turn, turns & 1u, &sh, p.err)) { ok = false; break; }
 #endif
         if (r == 0) TRACE(8 + 5 * qq, it);
         const float neg_m = -m_new;
+#if GCA_F32X2
+#pragma unroll
+        for (int e = 0; e < kTileK; e += 2) fma2_pair(sv[e], sv[e + 1], p.scale_log2, neg_m);
+#elif !GCA_FFMA_CHUNK
 #pragma unroll
         for (int e = 0; e < kTileK; ++e) sv[e] = fmaf(sv[e], p.scale_log2, neg_m);
+#endif
         float rs[8];
 #pragma unroll
         for (int a = 0; a < 8; ++a) rs[a] = 0.f;
-        uint32_t pk[kTileK / 2];
 #pragma unroll
         for (int chunk = 0; chunk < kTileK / 32; ++chunk) {
+          uint32_t pk[16];
+#if GCA_FFMA_CHUNK && !GCA_F32X2
+#pragma unroll
+          for (int e = 32 * chunk; e < 32 * chunk + 32; ++e) sv[e] = fmaf(sv[e], p.scale_log2, neg_m);
+#endif
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int e = 32 * chunk + 2 * c;
             const bool poly = c < GCA_POLY_PAIRS;
             const float e0 = poly ? exp2_poly(sv[e]) : ex2(sv[e]);
             const float e1 = poly ? exp2_poly(sv[e + 1]) : ex2(sv[e + 1]);
-            pk[16 * chunk + c] = pack_bf2(e0, e1);
+            pk[c] = pack_bf2(e0, e1);
+#if GCA_F32X2
+            add2_pair(rs[2 * (c & 3)], rs[2 * (c & 3) + 1], e0, e1);
+#else
             rs[2 * (c & 3)] += e0;
             rs[2 * (c & 3) + 1] += e1;
+#endif
           }
-          if (!GCA_LATE_PV) {
-            tmem_st16(t_row + kColP + 16 * chunk, reinterpret_cast<const float*>(pk + 16 * chunk));
+          tmem_st16(t_row + kColP + 16 * chunk, reinterpret_cast<const float*>(pk));
+          if (GCA_TURNS && chunk == kTileK / 32 - 1 - GCA_TURN_EARLY) {
+            if (GCA_TURN_WARP) {
+              __syncwarp();
+              if (lane == 0) mbar_arrive(their_turn);
+            } else {
+              mbar_arrive(their_turn);
+            }
           }
-          if (GCA_TURNS && chunk == kTileK / 32 - 1 - GCA_TURN_EARLY) mbar_arrive(&sh.turn[qq ^ 1]);
         }
         ++turns;
         if (r == 0) TRACE(9 + 5 * qq, it);
-        if (GCA_LATE_PV) {
-          // P V of the previous tile must be done before P is overwritten or O rescaled
-          if (j > j0) {
-            if (!sm_wait(&sh.pv_done[qq], (it - 1) & 1u, &sh, p.err)) { ok = false; break; }
-            tc_fence_after();
-          }
-          if (r == 0) TRACE(18 + qq, it);
-#pragma unroll
-          for (int chunk = 0; chunk < kTileK / 32; ++chunk) {
-            tmem_st16(t_row + kColP + 16 * chunk, reinterpret_cast<const float*>(pk + 16 * chunk));
-          }
-        }
         // Lazy rescale of O (rare): after the scores are dead, before P V(j) is issued.
         if (j > j0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
