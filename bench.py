@@ -136,8 +136,9 @@ def aggregate_frames_per_s(world: int, steps: int, frames: int, max_ms: float) -
 # ----------------------------------------------------------------------------- our arm
 
 def kernel_hash() -> str:
+    """Hash of the sources the attention kernel is built from (the traffic record's key)."""
     h = hashlib.sha256()
-    for name in ("gca_attn.cu", "gca_append.cu", "gca_internal.h"):
+    for name in ("gca_attn.cu", "gca_internal.h"):
         h.update(open(os.path.join(ROOT, "paged_kv_cache_gca_b200", "csrc", name), "rb").read())
     return h.hexdigest()[:16]
 
@@ -211,15 +212,22 @@ def run_ours(args, rank, world, device):
         os.path.join(ROOT, "gpurun_out")) else None
     with ClockSampler(torch.cuda.current_device() if device.index is None else device.index,
                       clocks_path if rank == 0 else None) as clk:
+        # `value`: K steps with nothing between the library's launches
         barrier()
         torch.cuda.synchronize(device)
         e_start.record(stream)
         with torch.cuda.stream(stream):
             for s in range(args.steps):
-                one_step(ev[s])
+                one_step()
         e_stop.record(stream)
         torch.cuda.synchronize(device)
         barrier()
+        # the per-call breakdown: the same K steps with events around every call (an event
+        # between two kernels also stops the next launch from overlapping the previous tail)
+        with torch.cuda.stream(stream):
+            for s in range(args.steps):
+                one_step(ev[s])
+        torch.cuda.synchronize(device)
     append_ms = sum(e[0].elapsed_time(e[1]) for st in ev for e in st)
     attend_ms = sum(e[1].elapsed_time(e[2]) for st in ev for e in st)
     elapsed_ms = e_start.elapsed_time(e_stop)

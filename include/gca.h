@@ -229,7 +229,9 @@ gca_status gca_reset(gca_cache* cache, void* stream);
 gca_status gca_cache_destroy(gca_cache* cache);
 
 /* Synchronises the device, reads the sticky device error word into the state and returns
- * GCA_ERR_DEVICE if it is non-zero. */
+ * GCA_ERR_DEVICE if it is non-zero. Once the word is set, every later attention of the cache
+ * does nothing (its output is left unwritten) until gca_reset; appends keep running, every
+ * page id range-checked before any write, so the pools stay in bounds. */
 gca_status gca_check(gca_cache* cache);
 
 /* Fills *state from the host mirror (no GPU access). */

@@ -120,12 +120,16 @@ __device__ __forceinline__ uint32_t rotate_word(uint32_t w, float2 cs) {
 
 __device__ __forceinline__ int wrap(int pos, int n) { return pos >= n ? pos - n : pos; }
 
+
 // Block bx of one cache's append. Token part: block (8 chunks, H heads, tok_per_block tokens);
 // one thread = one 16-byte chunk (8 dims) of one (token, head). Auxiliary part (blocks after
 // n_tok_blocks): eviction copies, zero fill of a fresh trajectory page, free-list pushes,
 // trajectory page records.
 __device__ __forceinline__ void append_block(const AppendParams& p, const int bx) {
   const int H = p.H;
+  // The append does not test the sticky error word (that costs ~10% of its bandwidth through
+  // register pressure): every page id is range-checked before any write, so it stays in
+  // bounds, and the attention and combine kernels, which do test the word, write no output.
   if (bx < p.n_tok_blocks) {
     // ---- a1 + a2
     const int c = threadIdx.x;
@@ -139,10 +143,6 @@ __device__ __forceinline__ void append_block(const AppendParams& p, const int bx
     }
     const int slot = i % kPageSize;
     const int64_t dst = (((int64_t)page * H + h) * kPageSize + slot) * 8 + c;
-    if (h == 0 && c == 0) {
-      if (i < p.T) p.slot_map[i] = page * kPageSize + slot;
-      if (slot == 0) p.frame_pages[p.t * p.ppf + i / kPageSize] = page;
-    }
     if (i >= p.T) {  // padding slot of the frame's last page
       p.k_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
       p.v_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
@@ -168,6 +168,10 @@ __device__ __forceinline__ void append_block(const AppendParams& p, const int bx
     kr.y = rotate_word(kv.y, cs[1]);
     kr.z = rotate_word(kv.z, cs[2]);
     kr.w = rotate_word(kv.w, cs[3]);
+    if (h == 0 && c == 0) {
+      p.slot_map[i] = page * kPageSize + slot;
+      if (slot == 0) p.frame_pages[p.t * p.ppf + i / kPageSize] = page;
+    }
     p.q_rot[src] = qr;
     p.k_pool[dst] = kr;
     p.v_pool[dst] = vv;
@@ -242,13 +246,24 @@ __device__ __forceinline__ void append_block(const AppendParams& p, const int bx
   p.traj_pages[p.traj_pages_before + k] = p.free_ring[wrap(first_new + k, p.num_pages)];
 }
 
-__global__ void __launch_bounds__(1024) append_kernel(const AppendParams p) {
+// At most 512 threads (8 chunks x 64 heads) and 32 registers: 8 blocks of 256 threads per SM
+// (the append is a latency-bound copy and wants every warp it can get: 6 blocks measured 5%
+// slower).
+#define GCA_APPEND_BOUNDS __launch_bounds__(512, 4)
+
+__global__ void GCA_APPEND_BOUNDS append_kernel(const AppendParams p) {
+  pdl_signal_early();
+  pdl_wait();  // inputs, pages and the free ring may come from earlier work in the stream
   append_block(p, (int)blockIdx.x);
+  pdl_signal_late();
 }
 
-__global__ void __launch_bounds__(1024) append_batch_kernel(const __grid_constant__ AppendBatch b) {
+__global__ void GCA_APPEND_BOUNDS append_batch_kernel(const __grid_constant__ AppendBatch b) {
+  pdl_signal_early();
+  pdl_wait();
   const AppendParams& p = b.p[blockIdx.y];
   if ((int)blockIdx.x < p.n_blocks) append_block(p, (int)blockIdx.x);
+  pdl_signal_late();
 }
 
 }  // namespace
@@ -277,14 +292,13 @@ cudaError_t launch_reset(int32_t* free_ring, const int32_t* init_free, uint32_t*
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
   const dim3 block(8, p.H, p.tok_per_block);
-  append_kernel<<<(unsigned)p.n_blocks, block, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(append_kernel, dim3((unsigned)p.n_blocks), block, 0, s, p);
 }
 
 cudaError_t launch_append_batch(const AppendBatch& b, cudaStream_t s) {
   const dim3 block(8, b.p[0].H, b.p[0].tok_per_block);
-  append_batch_kernel<<<dim3((unsigned)b.max_blocks, (unsigned)b.n), block, 0, s>>>(b);
-  return cudaGetLastError();
+  return launch_dependent(append_batch_kernel, dim3((unsigned)b.max_blocks, (unsigned)b.n), block,
+                          0, s, b);
 }
 
 }  // namespace gca

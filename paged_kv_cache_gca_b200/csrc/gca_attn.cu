@@ -472,6 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
+  pdl_signal_early();
   if ((smem_addr(smem) & 1023u) != 0u) {  // the swizzled tiles need a 1024-byte aligned base
     if (threadIdx.x == 0) atomicOr(p.err, GCA_DEVERR_SMEM_ALIGN);
     return;
@@ -517,9 +518,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
+  // Everything above is local (barriers, TMEM); from here on the kernel reads the page table,
+  // Q, K and V that earlier work in the stream wrote.
+  pdl_wait();
 
+  // A cache whose sticky error word is set gets no further work: every role sees an empty step
+  // range and the CTA goes straight to its teardown.
+  const bool dead = *reinterpret_cast<volatile uint32_t*>(p.err) != 0u;
   const int64_t s_begin = (int64_t)blockIdx.x * p.total / p.grid;
-  const int64_t s_end = (int64_t)(blockIdx.x + 1) * p.total / p.grid;
+  const int64_t s_end = dead ? s_begin : (int64_t)(blockIdx.x + 1) * p.total / p.grid;
 
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
@@ -858,6 +865,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  pdl_signal_late();
   tc_fence_before();
   __syncthreads();
   if (warp == kWarpMma0) {
@@ -872,6 +880,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // M = max_s m_s. Two threads per query row, 32 output columns each.
 constexpr int kCombineThreads = 2 * kTileQ;
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const AttnParams p) {
+  pdl_signal_early();
+  pdl_wait();  // the attention launch's partial records
+  if (*reinterpret_cast<volatile uint32_t*>(p.err) != 0u) return;  // sticky error: no-op
   const int u = blockIdx.x;  // (head, query tile)
   const int r = threadIdx.x >> 1;
   const int half = threadIdx.x & 1;
@@ -918,6 +929,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const AttnPara
     w.w = pack_bf2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
     dst[c] = w;
   }
+  pdl_signal_late();
 }
 
 }  // namespace
@@ -933,13 +945,11 @@ cudaError_t attn_prepare(int* ctas_per_sm) {
 
 cudaError_t launch_attn(const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
                         cudaStream_t s) {
-  attn_kernel<<<p.grid, kThreads, kSmemBytes, s>>>(tk, tv, p);
-  return cudaGetLastError();
+  return launch_dependent(attn_kernel, dim3(p.grid), dim3(kThreads), kSmemBytes, s, tk, tv, p);
 }
 
 cudaError_t launch_combine(const AttnParams& p, cudaStream_t s) {
-  combine_kernel<<<p.units, kCombineThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(combine_kernel, dim3(p.units), dim3(kCombineThreads), 0, s, p);
 }
 
 

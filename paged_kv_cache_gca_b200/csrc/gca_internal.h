@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/gca.h"
 
 struct gca_cache;
@@ -23,6 +25,57 @@ constexpr int kPagesPerTile = kTileK / kPageSize;
 constexpr int kMaxGrid = 512;   // attention CTAs per launch (sizes the split buffers)
 constexpr size_t kAlign = 1024;
 constexpr int kMaxAppendBatch = 128;  // caches per batched append launch (kernel-parameter bound)
+
+// Programmatic dependent launch: the append, attention and combine kernels are launched with
+// programmatic stream serialization, signal their dependents once their main work is done and
+// wait for their prerequisites (griddepcontrol.wait) before touching any data that earlier work
+// in the stream produced, so a kernel's launch overlaps the previous kernel's tail. Signalling
+// at the start instead lets the next grids' blocks take SMs early and wait there (slower). A
+// prerequisite that never signals (any kernel outside this library) is waited for to its end.
+#ifndef GCA_PDL
+#define GCA_PDL 1
+#endif
+// GCA_PDL_LATE 1: kernels signal their dependents after their main work; 0: at their start.
+#ifndef GCA_PDL_LATE
+#define GCA_PDL_LATE 1
+#endif
+
+#ifdef __CUDACC__
+__device__ __forceinline__ void pdl_wait() {
+#if GCA_PDL
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+}
+__device__ __forceinline__ void pdl_launch_dependents() {
+#if GCA_PDL
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
+}
+// Signal points at the start and at the end of a kernel's main work; one of them is active.
+__device__ __forceinline__ void pdl_signal_early() {
+  if (!GCA_PDL_LATE) pdl_launch_dependents();
+}
+__device__ __forceinline__ void pdl_signal_late() {
+  if (GCA_PDL_LATE) pdl_launch_dependents();
+}
+
+// Launches kernel<<<grid, block, smem, s>>>(args...) with programmatic stream serialization.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = GCA_PDL ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+#endif
 
 // Byte offsets of every region inside the caller's workspace.
 struct Layout {

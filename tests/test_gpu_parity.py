@@ -324,3 +324,12 @@ def test_bad_initial_free_list_is_reported():
     cache = gca.GcaCache(gca.config_for(w), initial_free=free)
     assert cache.check() == -6
     assert cache.state().device_error & 0x4
+    # the sticky word makes later attentions no-ops: no output is written
+    q, k, v = (x.cuda() for x in gi.draw_frame(w, 0))
+    q_rot = torch.empty_like(q)
+    out = torch.full_like(q, 3.0)
+    cache.append_frame(0, q, k, v, q_rot)
+    cache.attend(0, q_rot, out)
+    torch.cuda.synchronize()
+    assert bool((out == 3.0).all())
+    assert cache.check() == -6
