@@ -497,52 +497,59 @@ def run_batched_append(ring, device, stream, warm=16, timed=32):
 
 def run_e2e(args, w, cache, ring_host, device, stream, world):
     """Frames/s through the public API with inputs in pinned host memory: every frame's q, k, v
-    are copied host->device and its output device->host inside the timed region. Uploads and
-    downloads run on their own streams (one copy engine each way), ordered against the compute
-    stream by events, with three rotating input and output buffers: frame t+1's upload and
-    frame t-1's download overlap frame t's compute."""
+    are copied host->device and its output device->host inside the timed region. Copies move
+    chunks of 8 frames on their own streams (one copy engine each way), ordered against the
+    compute stream by events, with three rotating chunk buffers each way: chunk c+1's upload and
+    chunk c-1's download overlap chunk c's compute, and the 8 frames of a chunk run with no
+    stream operation between their launches."""
     T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    nframes = w.frames
+    C = 8 if nframes % 8 == 0 and w.ring % 8 == 0 else 1
     nbuf = 3
-    pinned = ring_host.pin_memory()
-    out_host = torch.empty((nbuf, T, H, D), dtype=torch.bfloat16).pin_memory()
-    inp = [torch.empty((3, T, H, D), dtype=torch.bfloat16, device=device) for _ in range(nbuf)]
+    nchunks = nframes // C
+    pinned = ring_host.pin_memory()  # [R, 3, T, H, D]
+    out_host = torch.empty((nbuf, C, T, H, D), dtype=torch.bfloat16).pin_memory()
+    inp = [torch.empty((C, 3, T, H, D), dtype=torch.bfloat16, device=device) for _ in range(nbuf)]
     q_rot = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
-    out = [torch.empty((T, H, D), dtype=torch.bfloat16, device=device) for _ in range(nbuf)]
+    out = [torch.empty((C, T, H, D), dtype=torch.bfloat16, device=device) for _ in range(nbuf)]
     h2d = torch.cuda.Stream(device=device)
     d2h = torch.cuda.Stream(device=device)
-    up = [torch.cuda.Event() for _ in range(nbuf)]        # input b uploaded
-    used = [torch.cuda.Event() for _ in range(nbuf)]      # input b consumed by the append
-    ready = [torch.cuda.Event() for _ in range(nbuf)]     # output b computed
-    down = [torch.cuda.Event() for _ in range(nbuf)]      # output b downloaded
-    nframes = w.frames
+    up = [torch.cuda.Event() for _ in range(nbuf)]        # input chunk b uploaded
+    used = [torch.cuda.Event() for _ in range(nbuf)]      # input chunk b consumed
+    ready = [torch.cuda.Event() for _ in range(nbuf)]     # output chunk b computed
+    down = [torch.cuda.Event() for _ in range(nbuf)]      # output chunk b downloaded
     steps = max(1, min(args.steps, 3))
     started = [False] * nbuf      # input buffer b has been uploaded into before
     downloading = [False] * nbuf  # output buffer b has a download issued (maybe in flight)
 
-    def upload(t):
-        b = t % nbuf
+    def upload(ci):
+        b = ci % nbuf
+        s0 = (ci * C) % w.ring
         with torch.cuda.stream(h2d):
             if started[b]:
-                h2d.wait_event(used[b])  # the append that read buffer b last has run
-            inp[b].copy_(pinned[t % w.ring], non_blocking=True)
+                h2d.wait_event(used[b])  # the chunk that read buffer b last has been appended
+            inp[b].copy_(pinned[s0:s0 + C], non_blocking=True)
             up[b].record(h2d)
         started[b] = True
 
     def step():
         cache.reset(stream=stream)
         upload(0)
-        if nframes > 1:
+        if nchunks > 1:
             upload(1)
-        for t in range(nframes):
-            b = t % nbuf
-            if t + 2 < nframes:
-                upload(t + 2)
+        for ci in range(nchunks):
+            b = ci % nbuf
+            if ci + 2 < nchunks:
+                upload(ci + 2)
             stream.wait_event(up[b])
-            cache.append_frame(t, inp[b][0], inp[b][1], inp[b][2], q_rot, stream=stream)
-            used[b].record(stream)
             if downloading[b]:
-                stream.wait_event(down[b])  # output b's previous frame has been downloaded
-            cache.attend(t, q_rot, out[b], stream=stream)
+                stream.wait_event(down[b])  # output b's previous chunk has been downloaded
+            for f in range(C):
+                t = ci * C + f
+                cache.append_frame(t, inp[b][f, 0], inp[b][f, 1], inp[b][f, 2], q_rot,
+                                   stream=stream)
+                cache.attend(t, q_rot, out[b][f], stream=stream)
+            used[b].record(stream)
             ready[b].record(stream)
             with torch.cuda.stream(d2h):
                 d2h.wait_event(ready[b])
