@@ -208,8 +208,7 @@ def run_ours(args, rank, world, device):
           for _ in range(args.steps)]
     e_start = torch.cuda.Event(enable_timing=True)
     e_stop = torch.cuda.Event(enable_timing=True)
-    clocks_path = os.path.join(ROOT, "gpurun_out", "bench_clocks.csv") if os.path.isdir(
-        os.path.join(ROOT, "gpurun_out")) else None
+    clocks_path = args.clocks_csv  # raw nvidia-smi samples, when asked for
     with ClockSampler(torch.cuda.current_device() if device.index is None else device.index,
                       clocks_path if rank == 0 else None) as clk:
         # `value`: K steps with nothing between the library's launches
@@ -676,6 +675,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="also write the raw nvidia-smi clock samples of the timed region here")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
