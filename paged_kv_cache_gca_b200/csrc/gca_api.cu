@@ -178,7 +178,7 @@ bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams
   p->n_tiles = (p->n_lp + kPagesPerTile - 1) / kPagesPerTile;
   p->n_qt = n_qt;
   p->units = cf.num_heads * n_qt;
-  p->n_pairs = (n_qt + 1) / 2;
+  p->n_pairs = (n_qt + kQPerCta - 1) / kQPerCta;
   p->units2 = cf.num_heads * p->n_pairs;
   p->total = (int64_t)p->units2 * p->n_tiles;
   int64_t gmax = std::min<int64_t>(kMaxGrid, (int64_t)c->sms * c->ctas_per_sm);

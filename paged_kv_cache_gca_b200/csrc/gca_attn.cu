@@ -112,7 +112,6 @@ __device__ long long g_trace[2][64][32];
 
 namespace {
 
-constexpr int kQPerCta = 2;        // query tiles per CTA (same head: they share every K/V tile)
 constexpr int kKStages = 3;        // K ring: a slot frees once both S = Q K^T are computed
 constexpr int kVStages = 3;        // V ring: a slot frees after both O += P V
 constexpr int kSoftmaxWarps = 4 * kQPerCta;
@@ -876,61 +875,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 
-// Merges the partial records of every split (head, query tile): weights 2^(m_s - M),
-// M = max_s m_s. Two threads per query row, 32 output columns each.
-constexpr int kCombineThreads = 2 * kTileQ;
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const AttnParams p) {
-  pdl_signal_early();
-  pdl_wait();  // the attention launch's partial records
-  if (*reinterpret_cast<volatile uint32_t*>(p.err) != 0u) return;  // sticky error: no-op
-  const int u = blockIdx.x;  // (head, query tile)
-  const int r = threadIdx.x >> 1;
-  const int half = threadIdx.x & 1;
-  const int h = u / p.n_qt;
-  const int qt = u % p.n_qt;
-  const int u2 = h * p.n_pairs + qt / kQPerCta;
-  const int qq = qt % kQPerCta;
-  const int64_t first = (int64_t)u2 * p.n_tiles;
-  const int64_t c0 = cta_of_step(first, p.total, p.grid);
-  const int64_t c1 = cta_of_step(first + p.n_tiles - 1, p.total, p.grid);
-  if (c0 == c1) return;
-  const int qi = qt * kTileQ + r;
-  if (qi >= p.T) return;
-  float M = -INFINITY;
-  for (int64_t c = c0; c <= c1; ++c) M = fmaxf(M, p.part_ml[part_slot(c, u2, qq) * kTileQ + r].x);
-  float acc[32];
-#pragma unroll
-  for (int a = 0; a < 32; ++a) acc[a] = 0.f;
-  float L = 0.f;
-  for (int64_t c = c0; c <= c1; ++c) {
-    const int64_t slot = part_slot(c, u2, qq);
-    const float2 ml = p.part_ml[slot * kTileQ + r];
-    const float w = ex2(ml.x - M);
-    L += w * ml.y;
-    const float4* src =
-        reinterpret_cast<const float4*>(p.part_o + (slot * kTileQ + r) * kHeadDim + 32 * half);
-#pragma unroll
-    for (int a = 0; a < 8; ++a) {
-      const float4 v = __ldcg(src + a);
-      acc[4 * a] += w * v.x;
-      acc[4 * a + 1] += w * v.y;
-      acc[4 * a + 2] += w * v.z;
-      acc[4 * a + 3] += w * v.w;
-    }
-  }
-  const float inv = 1.f / L;
-  uint4* dst = p.out + ((int64_t)qi * p.H + h) * 8 + 4 * half;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint4 w;
-    w.x = pack_bf2(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
-    w.y = pack_bf2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
-    w.z = pack_bf2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
-    w.w = pack_bf2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
-    dst[c] = w;
-  }
-  pdl_signal_late();
-}
 
 }  // namespace
 
@@ -948,9 +892,6 @@ cudaError_t launch_attn(const CUtensorMap& tk, const CUtensorMap& tv, const Attn
   return launch_dependent(attn_kernel, dim3(p.grid), dim3(kThreads), kSmemBytes, s, tk, tv, p);
 }
 
-cudaError_t launch_combine(const AttnParams& p, cudaStream_t s) {
-  return launch_dependent(combine_kernel, dim3(p.units), dim3(kCombineThreads), 0, s, p);
-}
 
 
 }  // namespace gca

@@ -21,6 +21,8 @@ constexpr int kMaxHeads = 64;
 constexpr int kMaxKeep = 64;
 constexpr int kTileQ = 128;     // query rows per attention tile
 constexpr int kTileK = 128;     // keys per attention tile (8 pages)
+constexpr int kQPerCta = 2;     // query tiles per attention CTA: a work unit is a pair of tiles
+                                // of one head (they share every K/V tile)
 constexpr int kPagesPerTile = kTileK / kPageSize;
 constexpr int kMaxGrid = 512;   // attention CTAs per launch (sizes the split buffers)
 constexpr size_t kAlign = 1024;
