@@ -135,6 +135,7 @@ bool compute_layout(const gca_config& c, Layout* L) {
   L->rope_t = take(8 * (size_t)c.max_frames * L->nt);
   L->rope_tok = take(8 * (size_t)T * (L->ny + L->nx));
   L->err = take(4);
+  L->kmax = take(4 * (size_t)c.num_heads);
   L->part_o = take(4 * (size_t)L->part_slots * kTileQ * kHeadDim);
   L->part_ml = take(8 * (size_t)L->part_slots * kTileQ);
   L->total = align_up(off, kAlign);
@@ -161,6 +162,7 @@ bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams
   p->frame_pages = reinterpret_cast<const int32_t*>(c->ws + L.frame_pages);
   p->traj_pages = reinterpret_cast<const int32_t*>(c->ws + L.traj_pages);
   p->err = reinterpret_cast<uint32_t*>(c->ws + L.err);
+  p->kmax = reinterpret_cast<const uint32_t*>(c->ws + L.kmax);
   if (q_rows <= 0) q_rows = L.T;
   const int32_t n_qt = (int32_t)((q_rows + kTileQ - 1) / kTileQ);
   p->T = (int32_t)q_rows;
@@ -294,7 +296,8 @@ gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t w
             cudaMemsetAsync(c->ws + L.v_pool, 0, (size_t)cfg->num_pages * page_bytes, s) ==
                 cudaSuccess &&
             cudaMemsetAsync(c->ws + L.seen, 0, 4 * (size_t)cfg->num_pages, s) == cudaSuccess &&
-            cudaMemsetAsync(c->ws + L.err, 0, 4, s) == cudaSuccess;
+            cudaMemsetAsync(c->ws + L.err, 0, 4, s) == cudaSuccess &&
+            cudaMemsetAsync(c->ws + L.kmax, 0, 4 * (size_t)cfg->num_heads, s) == cudaSuccess;
   if (ok) {
     InitParams ip;
     std::memset(&ip, 0, sizeof(ip));
@@ -370,6 +373,7 @@ gca_status prepare_append(gca_cache* c, int64_t t, int64_t rope_frame, uint32_t 
   p.rope_t = at<float2>(c, L.rope_t);
   p.rope_tok = at<float2>(c, L.rope_tok);
   p.err = at<uint32_t>(c, L.err);
+  p.kmax = at<uint32_t>(c, L.kmax);
   p.t = t;
   p.rope_frame = rope_frame;
   p.traj_len = c->traj_len;
@@ -527,7 +531,9 @@ gca_status gca_reset(gca_cache* c, void* stream) {
   const Layout& L = c->lay;
   if (launch_reset(at<int32_t>(c, L.free_ring), at<int32_t>(c, L.init_free),
                    at<uint32_t>(c, L.err), c->cfg.num_pages,
-                   static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+                   static_cast<cudaStream_t>(stream)) != cudaSuccess ||
+      cudaMemsetAsync(c->ws + L.kmax, 0, 4 * (size_t)c->cfg.num_heads,
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     return GCA_ERR_CUDA;
   }
   c->frames = 0;

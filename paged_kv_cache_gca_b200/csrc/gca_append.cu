@@ -175,6 +175,25 @@ __device__ __forceinline__ void append_block(const AppendParams& p, const int bx
     p.q_rot[src] = qr;
     p.k_pool[dst] = kr;
     p.v_pool[dst] = vv;
+    // The stored key's squared norm raises the head's running maximum: the attention bounds
+    // every score of a row by |q| * max|k| and skips its row max while that bound is below
+    // the running max + 2^8. Computed after the stores, when the q and v registers are free.
+    {
+      float ss = 0.f;
+      const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float a = bf_lo(kw[w]), b = bf_hi(kw[w]);
+        ss = fmaf(a, a, fmaf(b, b, ss));
+      }
+      // the 8 chunks of one (token, head) are 8 consecutive lanes
+      const unsigned lane = (threadIdx.x + 8u * (threadIdx.y + (unsigned)H * threadIdx.z)) & 31u;
+      const unsigned group = 0xffu << (lane & 24u);
+      ss += __shfl_xor_sync(group, ss, 1);
+      ss += __shfl_xor_sync(group, ss, 2);
+      ss += __shfl_xor_sync(group, ss, 4);
+      if (c == 0 && ss > __uint_as_float(p.kmax[h])) atomicMax(&p.kmax[h], __float_as_uint(ss));
+    }
     return;
   }
 

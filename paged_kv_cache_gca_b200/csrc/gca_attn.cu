@@ -682,7 +682,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qt = (u2 % p.n_pairs) * kQPerCta + qq;
       const int qi = qt * kTileQ + r;
 
-      // Q row -> shared memory, 128-byte swizzle (16-byte chunk c of row r at c ^ (r % 8))
+      // Q row -> shared memory, 128-byte swizzle (16-byte chunk c of row r at c ^ (r % 8)),
+      // and its squared norm
+      float q2 = 0.f;
       {
         const bool valid = qt < p.n_qt && qi < p.T;
         const uint4* src = p.q + ((int64_t)qi * p.H + h) * 8;
@@ -691,10 +693,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 8; ++c) {
           uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
           *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = v;
+          const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const float a = __uint_as_float(vw[w] << 16), b = __uint_as_float(vw[w] & 0xffff0000u);
+            q2 = fmaf(a, a, fmaf(b, b, q2));
+          }
         }
         fence_proxy_async_smem();
         mbar_arrive(&sh.q_full[qq]);
       }
+      // Every score of this row is at most |q| * max|k| (Cauchy-Schwarz; max|k| over every key
+      // appended to the cache, so it covers the keys this row sees). While that bound is within
+      // the lazy-rescale threshold of the running max, a tile's exact max cannot trigger a
+      // rescale, so the max pass is skipped and the same branch is taken. The factor covers
+      // rounding in the norms (a bound a hair too small only lets P reach 2^8 * (1 + eps)).
+      const float score_bound =
+          sqrtf(q2 * __uint_as_float(p.kmax[h])) * 1.01f * p.scale_log2;
 
       float m_run = -INFINITY;  // running row max, log2 units (scaled)
       float l_run = 0.f;        // running row sum relative to m_run
@@ -722,6 +737,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        float m_new = m_run, alpha = 1.f;
+        if (!(score_bound <= m_run + kRescaleThreshold)) {
         // row max: independent chains of 3-input max
         constexpr int kCh = GCA_MAX_CHAINS;
         float mx[kCh];
@@ -738,10 +755,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int a = 0; a < w; ++a) mx[a] = fmaxf(mx[a], mx[a + w]);
         }
         const float tile_max = mx[0] * p.scale_log2;
-        float m_new = m_run, alpha = 1.f;
         if (tile_max > m_run + kRescaleThreshold) {
           m_new = tile_max;
           alpha = ex2(m_run - m_new);
+        }
         }
         if (j > j0) {
           // P V of the previous tile must be done before P is overwritten or O rescaled

@@ -92,6 +92,7 @@ struct Layout {
   size_t rope_t;             // float2 (cos, sin) [max_frames][nt]: time band per frame
   size_t rope_tok;           // float2 (cos, sin) [T][ny + nx]: spatial bands per token
   size_t err;                // uint32 sticky device error word
+  size_t kmax;               // float [H] (as uint32 bits): max squared key norm ever appended
   size_t part_o;             // float [part_slots][128][64]
   size_t part_ml;            // float2 [part_slots][128]
   size_t total;
@@ -139,6 +140,7 @@ struct AppendParams {
   const float2* rope_t;
   const float2* rope_tok;
   uint32_t* err;
+  uint32_t* kmax;  // per head: max squared key norm (float bits), raised by every append
   int64_t t;           // cache frame (page-table row)
   int64_t rope_frame;  // RoPE time position (global frame index)
   int64_t traj_len;
@@ -175,6 +177,7 @@ struct AttnParams {
   const int32_t* frame_pages;
   const int32_t* traj_pages;
   uint32_t* err;
+  const uint32_t* kmax;  // per head: max squared key norm of everything appended
   int32_t T;  // query rows of the launch (T of one frame, or n * T for a joint prefill)
   int32_t H, ppf, last_len, num_pages;
   int32_t na_pages;      // anchor pages (visible anchor frames * ppf)
