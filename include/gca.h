@@ -22,7 +22,8 @@
  *     frame t-W (if >= A) is evicted; anchors (frames 0..A-1) are never evicted;
  *   - kept tokens of an evicted frame: K <= S: tokens 0..K-1; otherwise all S special tokens
  *     plus patches S + j*floor(P/(K-S)), j = 0..K-S-1;
- *   - attention scale 1/sqrt(D); no mask inside the current frame; frame-causal across frames;
+ *   - attention scale 1/sqrt(D); no mask inside the current frame; frame-causal across frames
+ *     (except the joint prefill of the first scale frames, gca_attend_prefill);
  *   - pages: FIFO free list; a frame takes ceil(T/page_size) pages (page-aligned); the
  *     trajectory pool is dense (page_size tokens per page) and never freed; the evicted
  *     frame's pages go back to the tail of the free list in row order.
@@ -71,9 +72,10 @@ typedef struct {
   int32_t anchor_frames; /* A >= 0 */
   int32_t window_frames; /* W >= 1, counts the current frame */
   int32_t keep_tokens;   /* K >= 0 tokens kept per evicted frame (0: no trajectory pool) */
-  int32_t max_frames;    /* frames one stream may append before gca_reset (RoPE table length) */
+  int32_t max_frames;    /* cache frames one stream may hold before gca_reset, and the RoPE
+                          * table length (every RoPE time position is < max_frames) */
   int32_t num_pages;     /* physical page capacity of the pool */
-  float rope_base;       /* RoPE theta (> 1) */
+  float rope_base;       /* RoPE theta (> 0, finite) */
 } gca_config;
 
 /* Host-mirrored counters and device addresses of a cache's state. Filling it never touches the
@@ -98,7 +100,8 @@ typedef struct {
   int32_t* kept_tokens;  /* int32 [K]: token indices an evicted frame keeps */
 } gca_state;
 
-/* Work description of the last gca_attend() call (host values, for measurement). */
+/* Work description of the last gca_attend() or gca_attend_prefill() call (host values, for
+ * measurement; gca_attend_noalloc does not update it). */
 typedef struct {
   int64_t frame_idx;
   int64_t visible_keys;  /* Nk(t): keys the frame's queries see */
