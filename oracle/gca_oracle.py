@@ -23,6 +23,10 @@ few tokens of each evicted frame [POOLS]; attention across frames is causal [GCT
 scale frames processed differently"]; a 12-frame window means 11 cached frames plus the current
 one [ABOT].
 
+Parity unpinned (by the pages): the conventions R1, R2 and R6 below are readings. The pins in
+the tests check that this code implements them as written (closed forms, invariants, hand-derived
+sequences), but no page fixes the conventions themselves.
+
 Readings where the pages are silent (each is listed in the design notes):
   R1 token order in a frame: [camera, registers, patches row-major over (grid_h, grid_w)].
   R2 RoPE band split d_y = d_x = 2*floor(D/6), d_t = D - d_y - d_x, order (t, y, x);
