@@ -6,6 +6,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import gca_inputs as gi
 import paged_kv_cache_gca_b200 as gca
@@ -114,3 +115,29 @@ def test_create_rejects_bad_arguments_before_touching_cuda(L):
     assert L.gca_append_frames(None, 1, idx, one, one, one, one, None) == -1
     assert L.gca_append_frames(one, 1, None, one, one, one, one, None) == -1
     assert L.gca_append_frames(nul, 1, idx, one, one, one, one, None) == -1
+
+
+def test_binding_routes_each_call_to_its_entry_point(L):
+    # a cache object whose handle is NULL: the library rejects every call before touching CUDA,
+    # and the error names the entry point the binding chose
+    cache = gca.GcaCache.__new__(gca.GcaCache)
+    cache.handle = None
+    x = torch.zeros(4, dtype=torch.bfloat16)
+
+    def where(fn, *a, **kw):
+        with pytest.raises(gca.GcaError) as e:
+            fn(*a, **kw)
+        assert e.value.status == -1
+        return str(e.value).split(":")[0]
+
+    assert where(cache.append_frame, 0, x, x, x, x, stream=0) == "gca_append_frame"
+    assert where(cache.append_frame, 0, x, x, x, x, stream=0, transient=True) == \
+        "gca_append_frame_ex"
+    assert where(cache.append_frame, 0, x, x, x, x, stream=0, rope_frame=3) == \
+        "gca_append_frame_ex"
+    assert where(cache.attend, 0, x, x, stream=0) == "gca_attend"
+    assert where(cache.attend_prefill, 2, x, x, stream=0) == "gca_attend_prefill"
+    assert where(cache.rollback, 0) == "gca_rollback_last_frame"
+    assert where(cache.reset, stream=0) == "gca_reset"
+    assert where(gca.gca_append_frames, [None], [0], [1], [1], [1], [1], 0) == \
+        "gca_append_frames"
