@@ -630,7 +630,8 @@ def oracle_frames_per_s(w: gi.Workload, sample_frames):
     est = t_book + t_att * all_pairs / sampled_pairs
     return w.frames / est, {
         "bookkeeping_s": round(t_book, 3), "attention_s_sampled": round(t_att, 3),
-        "estimated_stream_s": round(est, 3)}
+        "estimated_stream_s": round(est, 3), "nproc": os.cpu_count(),
+        "torch_threads": torch.get_num_threads()}
 
 
 def run_reference(args):
