@@ -28,7 +28,9 @@
  *     trajectory pool is dense (page_size tokens per page) and never freed; the evicted
  *     frame's pages go back to the tail of the free list in row order.
  *
- * Tensors are raw device pointers, bf16, contiguous, token-major "NHD": [T][H][D].
+ * Tensors are raw device pointers, bf16, contiguous, token-major "NHD": [T][H][D], 16-byte
+ * aligned (the kernels move them in 16-byte vectors; a misaligned pointer is rejected with
+ * GCA_ERR_INVALID_ARG). A device initial free list must be 4-byte aligned.
  * Streams are cudaStream_t passed as void* (NULL = legacy default stream).
  * Calls that enqueue work never synchronise; only gca_check() does.
  * Supported sizes: head_dim 64, page_size 16, 1 <= num_heads <= 64, keep_tokens <= 64.

@@ -214,6 +214,10 @@ T* at(gca_cache* c, size_t off) {
   return reinterpret_cast<T*>(c->ws + off);
 }
 
+// Device tensors are read and written as 16-byte vectors; a misaligned pointer is rejected on
+// the host instead of faulting on the device.
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 bool on_cache_device(const gca_cache* c) {
   int d = -1;
   return cudaGetDevice(&d) == cudaSuccess && d == c->device;
@@ -258,6 +262,7 @@ gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t w
       ws_bytes < L.total) {
     return GCA_ERR_INVALID_ARG;
   }
+  if ((reinterpret_cast<uintptr_t>(dev_initial_free_list) & 3u) != 0) return GCA_ERR_INVALID_ARG;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GCA_ERR_CUDA;
   int sms = 0;
@@ -340,6 +345,9 @@ gca_status prepare_append(gca_cache* c, int64_t t, int64_t rope_frame, uint32_t 
                           const void* q, const void* k, const void* v, void* q_rot_out,
                           AppendParams* out) {
   if (!c || !q || !k || !v || !q_rot_out) return GCA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_rot_out)) {
+    return GCA_ERR_INVALID_ARG;
+  }
   if ((flags & ~(uint32_t)GCA_APPEND_TRANSIENT) != 0u) return GCA_ERR_INVALID_ARG;
   if (t != c->frames || c->transient) return GCA_ERR_FRAME_ORDER;
   if (t >= c->cfg.max_frames) return GCA_ERR_INVALID_ARG;
@@ -509,7 +517,7 @@ gca_status enqueue_attention(gca_cache* c, int64_t t, int64_t q_rows, const void
 }  // namespace
 
 gca_status gca_attend(gca_cache* c, int64_t t, const void* q_rot, void* out, void* stream) {
-  if (!c || !q_rot || !out) return GCA_ERR_INVALID_ARG;
+  if (!c || !q_rot || !out || !aligned16(q_rot) || !aligned16(out)) return GCA_ERR_INVALID_ARG;
   if (c->frames == 0 || t != c->frames - 1) return GCA_ERR_FRAME_ORDER;
   if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;
   return enqueue_attention(c, t, 0, q_rot, out, stream);
@@ -517,7 +525,7 @@ gca_status gca_attend(gca_cache* c, int64_t t, const void* q_rot, void* out, voi
 
 gca_status gca_attend_prefill(gca_cache* c, int32_t n, const void* q_rot, void* out,
                               void* stream) {
-  if (!c || !q_rot || !out) return GCA_ERR_INVALID_ARG;
+  if (!c || !q_rot || !out || !aligned16(q_rot) || !aligned16(out)) return GCA_ERR_INVALID_ARG;
   if (n < 1 || n > c->cfg.anchor_frames) return GCA_ERR_INVALID_ARG;
   if (c->frames != n || c->transient) return GCA_ERR_FRAME_ORDER;
   if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;

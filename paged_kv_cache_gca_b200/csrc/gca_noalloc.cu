@@ -59,6 +59,10 @@ using namespace gca;
 extern "C" gca_status gca_attend_noalloc(gca_cache* c, int64_t t, const void* q_rot, void* out,
                                          void* stream) {
   if (!c || !q_rot || !out) return GCA_ERR_INVALID_ARG;
+  // 16-byte vector accesses: a misaligned tensor is rejected here, not faulted on the device
+  if (((reinterpret_cast<uintptr_t>(q_rot) | reinterpret_cast<uintptr_t>(out)) & 15u) != 0) {
+    return GCA_ERR_INVALID_ARG;
+  }
   if (c->frames == 0 || t != c->frames - 1) return GCA_ERR_FRAME_ORDER;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != c->device) return GCA_ERR_INVALID_ARG;

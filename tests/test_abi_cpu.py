@@ -95,6 +95,8 @@ def test_create_rejects_bad_arguments_before_touching_cuda(L):
     assert L.gca_cache_create(ctypes.byref(cfg), None, n, None, None, ctypes.byref(h)) == -1
     assert L.gca_cache_create(ctypes.byref(cfg), 1024 + 16, n, None, None, ctypes.byref(h)) == -1
     assert L.gca_cache_create(ctypes.byref(cfg), 1024, n - 1, None, None, ctypes.byref(h)) == -1
+    # a misaligned device free list is rejected before any CUDA call
+    assert L.gca_cache_create(ctypes.byref(cfg), 1024, n, 4096 + 2, None, ctypes.byref(h)) == -1
     assert h.value is None
     # calls on a null handle
     assert L.gca_append_frame(None, 0, 1, 1, 1, 1, None) == -1
