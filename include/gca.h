@@ -192,7 +192,8 @@ gca_status gca_append_frames(gca_cache* const* caches, int32_t n, const int64_t*
 /* Attention of the last appended frame's queries over the cache (pages' compute_attention):
  * out[i][h] = softmax_j(q_rot[i][h] . k_j[h] / sqrt(D)) v_j[h] over the anchor, window and
  * trajectory keys visible at frame frame_idx (which must be the last appended frame).
- * q_rot: device bf16 [T][H][D] from gca_append_frame; out: device bf16 [T][H][D].
+ * q_rot: device bf16 [T][H][D] from gca_append_frame; out: device bf16 [T][H][D], not
+ * overlapping q_rot (GCA_ERR_INVALID_ARG: CTAs still read queries while others write rows).
  * One tcgen05 attention launch, plus one combine launch when the key range is split. */
 gca_status gca_attend(gca_cache* cache, int64_t frame_idx, const void* q_rot, void* out,
                       void* stream);
@@ -202,7 +203,8 @@ gca_status gca_attend(gca_cache* cache, int64_t frame_idx, const void* q_rot, vo
  * attend over every token of those frames, with no mask across frames (pages: the scale frames
  * are processed jointly with bidirectional attention, then streaming switches to causal;
  * Streaming Inference API, FAQ on scale frames). q_rot: device bf16 [n*T][H][D], the q_rot
- * outputs of the n appends back to back (frame-major); out: device bf16 [n*T][H][D]. One
+ * outputs of the n appends back to back (frame-major); out: device bf16 [n*T][H][D], not
+ * overlapping q_rot (GCA_ERR_INVALID_ARG). One
  * attention launch (+ one combine launch when split). GCA_ERR_INVALID_ARG unless
  * 1 <= n <= anchor_frames; GCA_ERR_FRAME_ORDER unless exactly n frames are appended (and no
  * transient frame is pending). */

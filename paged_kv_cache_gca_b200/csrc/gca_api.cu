@@ -218,6 +218,13 @@ T* at(gca_cache* c, size_t off) {
 // the host instead of faulting on the device.
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// [a, a + bytes) and [b, b + bytes) overlap: an attention output over its own queries would
+// race (CTAs still load a unit's Q rows while others write output rows).
+bool overlaps(const void* a, const void* b, size_t bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + bytes && y < x + bytes;
+}
+
 bool on_cache_device(const gca_cache* c) {
   int d = -1;
   return cudaGetDevice(&d) == cudaSuccess && d == c->device;
@@ -520,6 +527,8 @@ gca_status gca_attend(gca_cache* c, int64_t t, const void* q_rot, void* out, voi
   if (!c || !q_rot || !out || !aligned16(q_rot) || !aligned16(out)) return GCA_ERR_INVALID_ARG;
   if (c->frames == 0 || t != c->frames - 1) return GCA_ERR_FRAME_ORDER;
   if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;
+  const size_t bytes = (size_t)c->lay.T * c->cfg.num_heads * kHeadDim * 2;
+  if (overlaps(q_rot, out, bytes)) return GCA_ERR_INVALID_ARG;
   return enqueue_attention(c, t, 0, q_rot, out, stream);
 }
 
@@ -529,6 +538,8 @@ gca_status gca_attend_prefill(gca_cache* c, int32_t n, const void* q_rot, void* 
   if (n < 1 || n > c->cfg.anchor_frames) return GCA_ERR_INVALID_ARG;
   if (c->frames != n || c->transient) return GCA_ERR_FRAME_ORDER;
   if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;
+  const size_t bytes = (size_t)n * c->lay.T * c->cfg.num_heads * kHeadDim * 2;
+  if (overlaps(q_rot, out, bytes)) return GCA_ERR_INVALID_ARG;
   // frames 0..n-1 are all anchors (n <= A), so frame n-1's key set is every token of them
   return enqueue_attention(c, n - 1, (int64_t)n * c->lay.T, q_rot, out, stream);
 }

@@ -66,6 +66,11 @@ extern "C" gca_status gca_attend_noalloc(gca_cache* c, int64_t t, const void* q_
   if (c->frames == 0 || t != c->frames - 1) return GCA_ERR_FRAME_ORDER;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != c->device) return GCA_ERR_INVALID_ARG;
+  {  // an output over its own queries would race
+    const uintptr_t x = reinterpret_cast<uintptr_t>(q_rot), y = reinterpret_cast<uintptr_t>(out);
+    const size_t bytes = (size_t)c->lay.T * c->cfg.num_heads * kHeadDim * 2;
+    if (x < y + bytes && y < x + bytes) return GCA_ERR_INVALID_ARG;
+  }
   // The partial records of one call must fit the array (at least one CTA per work unit).
   AttnParams p;
   bool split = false;
