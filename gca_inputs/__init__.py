@@ -4,8 +4,9 @@ This module is shared by the CUDA path's tests/bench and by the CPU oracle. It h
 shapes, seeds and random draws only: no RoPE, no paging, no attention arithmetic.
 
 Workload shapes follow the pages' streaming setup:
-  * LingBot-Map at 518x378 with patch 14 gives a 37x27 patch grid (999 patches), plus a
-    camera token and register tokens ("How GCT's Anchor-Pose-Trajectory Pools Make
+  * LingBot-Map at 518x378 with patch 14: the size is read as width x height, as image
+    sizes are usually quoted, so a frame is 27 patch rows x 37 patch columns (999 patches),
+    plus a camera token and register tokens ("How GCT's Anchor-Pose-Trajectory Pools Make
     Monocular 3D Tractable", first paragraph; GCT deep-dive page, "Practical Usage
     Example": img_size 518, patch_size 14, embed_dim 1024 = 16 heads x 64).
   * Sliding windows of 16-64 frames (same news page, pool list), the 320-view RoPE
@@ -88,27 +89,27 @@ WORKLOADS = {
         seed=0, value_scale=1.0, permuted_free_list=True, ring=6, num_pages=24,
         max_frames=64),
     "w16_320": Workload(
-        name="w16_320", num_heads=16, head_dim=64, page_size=16, grid_h=37, grid_w=27,
+        name="w16_320", num_heads=16, head_dim=64, page_size=16, grid_h=27, grid_w=37,
         num_special=5, anchor_frames=1, window_frames=16, keep_tokens=12, frames=320,
         seed=1, value_scale=0.125, permuted_free_list=False, ring=64, num_pages=1400,
         max_frames=320),
     "w64_1000": Workload(
-        name="w64_1000", num_heads=16, head_dim=64, page_size=16, grid_h=37, grid_w=27,
+        name="w64_1000", num_heads=16, head_dim=64, page_size=16, grid_h=27, grid_w=37,
         num_special=5, anchor_frames=1, window_frames=64, keep_tokens=12, frames=1000,
         seed=2, value_scale=0.125, permuted_free_list=True, ring=64, num_pages=4900,
         max_frames=1000),
     "w32_10k": Workload(
-        name="w32_10k", num_heads=16, head_dim=64, page_size=16, grid_h=37, grid_w=27,
+        name="w32_10k", num_heads=16, head_dim=64, page_size=16, grid_h=27, grid_w=37,
         num_special=5, anchor_frames=1, window_frames=32, keep_tokens=12, frames=10000,
         seed=3, value_scale=0.125, permuted_free_list=False, ring=64, num_pages=9650,
         max_frames=10000),
     "stack24x4": Workload(
-        name="stack24x4", num_heads=16, head_dim=64, page_size=16, grid_h=37, grid_w=27,
+        name="stack24x4", num_heads=16, head_dim=64, page_size=16, grid_h=27, grid_w=37,
         num_special=5, anchor_frames=0, window_frames=12, keep_tokens=0, frames=500,
         seed=4, value_scale=0.125, permuted_free_list=False, ring=64, num_pages=832,
         max_frames=500, num_layers=24, num_streams=4, rope_base_varies_by_layer=True),
     "scale8": Workload(
-        name="scale8", num_heads=16, head_dim=64, page_size=16, grid_h=37, grid_w=27,
+        name="scale8", num_heads=16, head_dim=64, page_size=16, grid_h=27, grid_w=37,
         num_special=5, anchor_frames=8, window_frames=16, keep_tokens=12, frames=48,
         seed=5, value_scale=0.125, permuted_free_list=True, ring=64, num_pages=1650,
         max_frames=48),

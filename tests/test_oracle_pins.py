@@ -198,13 +198,54 @@ def test_rope_bands_touch_their_own_dims():
 
 
 def test_token_positions_row_major_after_special_tokens():
-    pos = orc.token_positions(9, 5, 37, 27)
+    pos = orc.token_positions(9, 5, 27, 37)
     assert pos.shape == (1004, 3)
     assert (pos[:, 0] == 9).all()
     assert (pos[:5, 1:] == 0).all()
     assert tuple(pos[5]) == (9, 1, 1)
-    assert tuple(pos[5 + 27]) == (9, 2, 1)
-    assert tuple(pos[-1]) == (9, 37, 27)
+    assert tuple(pos[5 + 36]) == (9, 1, 37)
+    assert tuple(pos[5 + 37]) == (9, 2, 1)
+    assert tuple(pos[-1]) == (9, 27, 37)
+
+
+# Angles of the RoPE reading written out by hand (3D RoPE of the GCT page: bands t, y, x of
+# 24, 20, 20 dims at head_dim 64; pair j of a band of width d turns by pos * base^(-2j/d)).
+# The column of pair j is j in the time band, 12 + j in the y band and 22 + j in the x band.
+# Each value is the exponent simplified by hand, e.g. 10000^(-2*1/24) = 10^(-1/3).
+ROPE_HAND_VALUES = [
+    # (base, (t, y, x), column, angle)
+    (10000.0, (7, 3, 11), 0, 7.0),                      # t * 10000^0
+    (10000.0, (7, 3, 11), 1, 3.2491121835289450),       # 7 * 10^(-1/3)
+    (10000.0, (7, 3, 11), 6, 0.07),                     # 7 * 10000^(-12/24) = 7 * 10^-2
+    (10000.0, (7, 3, 11), 11, 7 * 2.1544346900318823e-4),  # 7 * 10^(-11/3)
+    (10000.0, (7, 3, 11), 12, 3.0),                     # y * 10000^0
+    (10000.0, (7, 3, 11), 15, 0.18928720334405799),     # 3 * 10000^(-6/20) = 3 * 10^(-1.2)
+    (10000.0, (7, 3, 11), 17, 0.03),                    # 3 * 10000^(-10/20) = 3 * 10^-2
+    (10000.0, (7, 3, 11), 22, 11.0),                    # x * 10000^0
+    (10000.0, (7, 3, 11), 24, 1.7433825117072247),      # 11 * 10000^(-4/20) = 11 * 10^(-0.8)
+    (10000.0, (7, 3, 11), 31, 0.0027630750746605374),   # 11 * 10000^(-18/20) = 11 * 10^(-3.6)
+    (500.0, (7, 3, 11), 6, 0.31304951684997057),        # 7 * 500^(-1/2)
+    (500.0, (7, 3, 11), 17, 0.13416407864998738),       # 3 * 500^(-1/2)
+    (500.0, (7, 3, 11), 27, 0.49193495504995373),       # 11 * 500^(-1/2)
+    (500.0, (7, 3, 11), 3, 7 * 0.21147425268811282),    # 7 * 500^(-1/4)
+]
+
+
+@pytest.mark.parametrize("base,pos,col,angle", ROPE_HAND_VALUES)
+def test_rope_angles_match_hand_values(base, pos, col, angle):
+    ang = orc.rope_angles(np.array([pos], dtype=np.int64), 64, base)
+    assert ang.shape == (1, 32)
+    assert abs(ang[0, col] - angle) <= 1e-13 * max(1.0, abs(angle))
+
+
+def test_rope_rotation_of_a_unit_pair_by_hand():
+    # the time-band pair j = 6 of a token at t = 7 turns (1, 0) into (cos 0.07, sin 0.07)
+    x = np.zeros((1, 1, 64))
+    x[0, 0, 12] = 1.0
+    out = orc.rotate_pairs(x, orc.rope_angles(np.array([[7, 3, 11]]), 64, 10000.0))
+    assert abs(out[0, 0, 12] - 0.99755100025327959) < 1e-14   # cos(0.07)
+    assert abs(out[0, 0, 13] - 0.06994284733753277) < 1e-14   # sin(0.07)
+    assert np.count_nonzero(out[0, 0]) == 2
 
 
 # ------------------------------------------------------------------ pools and kept tokens
@@ -247,10 +288,14 @@ def test_pool_sizes_at_the_last_frame():
 
 def test_pages_print_the_shapes():
     facts = json.load(open(os.path.join(GOLDEN, "pages_facts.json")))
-    (wpx, hpx), p = facts["image_hw"]["value"], facts["patch_size"]["value"]
+    (wpx, hpx), p = facts["image_width_height"]["value"], facts["patch_size"]["value"]
     gw_, gh_ = wpx // p, hpx // p
+    assert (gh_, gw_) == (27, 37) and gh_ * gw_ == 999
+    # every 518x378 workload lays its patches out as 27 rows x 37 columns
+    for name, wl in gi.WORKLOADS.items():
+        if wl.tokens_per_frame == 1004:
+            assert (wl.grid_h, wl.grid_w) == (gh_, gw_), name
     w = gi.workload("w16_320")
-    assert (gh_, gw_) == (27, 37) and gh_ * gw_ == 999 == w.grid_h * w.grid_w
     assert facts["embed_dim"]["value"] == w.num_heads * w.head_dim
     # per-frame context growth: T tokens (full causal) vs K kept tokens
     ratio = w.tokens_per_frame / w.keep_tokens
