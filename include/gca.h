@@ -137,7 +137,8 @@ gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t w
  * RoPE on q and k, k_rot and v scattered into freshly popped pages, q_rot written for
  * gca_attend, and the frame that leaves the window evicted (kept tokens copied to the
  * trajectory tail, its pages pushed back to the free list) -- one kernel launch.
- * q, k, v: device bf16 [T][H][D]; q_rot_out: device bf16 [T][H][D] (may alias q).
+ * q, k, v: device bf16 [T][H][D]; q_rot_out: device bf16 [T][H][D]: it may be q itself, but
+ * any other overlap with q, k or v is rejected (GCA_ERR_INVALID_ARG).
  * frame_idx must equal the number of frames appended since create/reset
  * (GCA_ERR_FRAME_ORDER) and be < max_frames. The page budget is checked on the host from
  * mirrored counts: GCA_ERR_OUT_OF_PAGES returns with nothing enqueued. */
@@ -218,7 +219,9 @@ gca_status gca_attend_prefill(gca_cache* cache, int32_t n, const void* q_rot, vo
  * It allocates nothing. Its scratch -- the split-KV partial records -- lives in a 16 MiB array
  * inside this library, which every GPU that loads the library holds until the process exits.
  * The first call on a device looks up that array's device address (cudaGetSymbolAddress) with
- * the device current; make that first call before any stream capture. All calls share the one
+ * the device current; make that first call before any stream capture. The address is kept with
+ * the CUDA context it was taken in and looked up again when the context changes (for example
+ * after a cudaDeviceReset). All calls share the one
  * array and it keeps the last call's contents (every slot read is written earlier in the same
  * call): calls whose kernels overlap on the GPU race on it, so order them (one stream, or
  * events). The array holds 496 partial records of 128 query rows; a launch over num_heads *

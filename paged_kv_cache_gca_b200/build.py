@@ -22,6 +22,17 @@ def nvcc() -> str:
     return "nvcc"
 
 
+def build_command(verbose: bool = False, out: str | None = None) -> list[str]:
+    """The nvcc command line that builds the library (sm_100a only)."""
+    srcs = [os.path.join(CSRC, s) for s in SOURCES]
+    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+           "-cudart", "static", "-o", (LIB if out is None else out) + ".tmp", *srcs, "-ldl",
+           "-lrt", "-lpthread"]
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+    return cmd
+
+
 def build(verbose: bool = False, force: bool = False) -> str:
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
     deps = srcs + [os.path.join(CSRC, "gca_internal.h"),
@@ -30,10 +41,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
         lib_t = os.path.getmtime(LIB)
         if all(os.path.getmtime(d) <= lib_t for d in deps):
             return LIB
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-cudart", "static", "-o", LIB + ".tmp", *srcs, "-ldl", "-lrt", "-lpthread"]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
+    cmd = build_command(verbose)
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)

@@ -355,6 +355,16 @@ gca_status prepare_append(gca_cache* c, int64_t t, int64_t rope_frame, uint32_t 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_rot_out)) {
     return GCA_ERR_INVALID_ARG;
   }
+  {
+    // Each thread reads its own chunk of q, k, v and writes the same chunk of q_rot, so q_rot
+    // may be q itself; any other overlap with q, k or v would let a thread overwrite a chunk
+    // another thread has yet to read.
+    const size_t bytes = (size_t)c->lay.T * c->cfg.num_heads * kHeadDim * 2;
+    if ((q_rot_out != q && overlaps(q_rot_out, q, bytes)) || overlaps(q_rot_out, k, bytes) ||
+        overlaps(q_rot_out, v, bytes)) {
+      return GCA_ERR_INVALID_ARG;
+    }
+  }
   if ((flags & ~(uint32_t)GCA_APPEND_TRANSIENT) != 0u) return GCA_ERR_INVALID_ARG;
   if (t != c->frames || c->transient) return GCA_ERR_FRAME_ORDER;
   if (t >= c->cfg.max_frames) return GCA_ERR_INVALID_ARG;

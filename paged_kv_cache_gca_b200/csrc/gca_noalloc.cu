@@ -34,20 +34,49 @@ constexpr int kMaxDevices = 64;
 __device__ __align__(256) unsigned char g_attend_scratch[kNoallocScratchBytes];
 
 // Device address of g_attend_scratch per device. In host code the symbol's name is only a
-// host-side stand-in, so the address is looked up once per device, with that device current.
+// host-side stand-in, so the address is looked up with the device current, once per device and
+// CUDA context: the address is cached next to the context it was taken in and looked up again
+// when the device's current context is a different one (after a cudaDeviceReset, or when the
+// caller destroyed and re-created the primary context), so a stale address is never used.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    }
+  });
+  return fn;
+}
+
+struct ScratchEntry {
+  CUcontext ctx;
+  void* addr;
+};
 std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+ScratchEntry g_scratch[kMaxDevices] = {};
 
 cudaError_t scratch_address(int dev, void** out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  CtxGetCurrentFn get_ctx = ctx_get_current();
+  if (!get_ctx) return cudaErrorNotSupported;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorContextIsDestroyed;
+  if (!ctx || !g_scratch[dev].addr || g_scratch[dev].ctx != ctx) {
     void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_attend_scratch);
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_attend_scratch);  // also makes a context
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorContextIsDestroyed;
+    g_scratch[dev].ctx = ctx;
+    g_scratch[dev].addr = p;
   }
-  *out = g_scratch_addr[dev];
+  *out = g_scratch[dev].addr;
   return cudaSuccess;
 }
 

@@ -308,6 +308,17 @@ def test_host_detected_errors():
     with pytest.raises(gca.GcaError) as e:
         cache.attend(0, q_rot, out)
     assert e.value.status == -3
+    # q_rot_out may be q itself, but no other overlap with q, k or v: a shifted overlap would
+    # let one thread overwrite a chunk another has yet to read
+    big = torch.empty((3 * w.tokens_per_frame + 8, w.num_heads, w.head_dim),
+                      dtype=torch.bfloat16, device="cuda")
+    T = w.tokens_per_frame
+    qb, kb = big[:T], big[T:2 * T]
+    for bad in (big[1:T + 1], big[T:2 * T], big[T - 1:2 * T - 1]):
+        with pytest.raises(gca.GcaError) as e:
+            cache.append_frame(0, qb, kb, v, bad)
+        assert e.value.status == -1
+    assert cache.state().frames_appended == 0
     cache.append_frame(0, q, k, v, q_rot)
     cache.append_frame(1, q, k, v, q_rot)
     # 12 pages, 5 per frame: the third frame does not fit

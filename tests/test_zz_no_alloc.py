@@ -34,20 +34,28 @@ def test_noalloc_matches_attend_on_two_calls_in_a_row():
     ref = torch.empty_like(q_rot)
     got = [torch.empty_like(q_rot), torch.empty_like(q_rot)]
     stream = torch.cuda.current_stream().cuda_stream
-    checked = 0
+    checked = split = 0
     for t in range(w.frames):
         q, k, v = ring[t % w.ring]
         cache.append_frame(t, q, k, v, q_rot)
         if t in (0, 17, w.frames - 1):
             cache.attend(t, q_rot, ref)
+            # gca_attend_noalloc plans the same launch (the same grid here: the scratch holds
+            # every record this config needs), so gca_attend's info tells whether the key
+            # ranges were split, i.e. whether the call went through the library's array
+            split += cache.attend_info().split
+            torch.cuda.synchronize()
+            free_before = torch.cuda.mem_get_info()[0]
             for g in got:  # two calls in a row share (and reuse) the library's scratch array
                 gca.gca_attend_noalloc(cache.handle, t, q_rot.data_ptr(), g.data_ptr(), stream)
             torch.cuda.synchronize()
+            assert torch.cuda.mem_get_info()[0] == free_before  # nothing was allocated
             r = ref.double().cpu().numpy()
             for g in got:
                 check_attention(g.double().cpu().numpy(), r, f"noalloc t={t}")
             checked += 1
     assert checked == 3
+    assert split >= 2  # frames 17 and 47 split their key ranges: the combine read the array
     assert cache.check() == 0
 
 
