@@ -17,6 +17,12 @@ Workload shapes follow the pages' streaming setup:
 Per-frame draws: q, k, v ~ N(0, 1) * scale in fp32, rounded to bf16. Frame t of a
 stream takes its data from ring slot t mod ring, so a long stream reuses a bounded set
 of distinct frames (RoPE positions still differ per frame).
+
+Needles (optional, for tests of the online softmax's rescale path): every query gets a
+common component q_gain * u_h along a fixed unit direction u_h per head, and in ring slots
+with slot % needle_every == needle_slot the keys of token 0 (the camera token, which an
+evicted frame keeps in the trajectory pool) and of the frame's last token (its last page)
+are set to k_gain * u_h. Those keys then score far above all others, late in the key order.
 """
 from __future__ import annotations
 
@@ -34,6 +40,7 @@ __all__ = [
     "draw_ring",
     "initial_free_list",
     "rope_base_for_layer",
+    "needle_directions",
 ]
 
 
@@ -60,6 +67,10 @@ class Workload:
     num_layers: int = 1  # independent caches per stream (stack stress)
     num_streams: int = 1  # concurrent streams
     rope_base_varies_by_layer: bool = False
+    needle_every: int = 0  # 0: no needles; else slots with slot % needle_every == needle_slot
+    needle_slot: int = 0
+    needle_q_gain: float = 0.0
+    needle_k_gain: float = 0.0
 
     @property
     def tokens_per_frame(self) -> int:
@@ -129,6 +140,13 @@ def frame_seed(seed: int, slot: int) -> int:
     return seed * 1_000_003 + slot
 
 
+def needle_directions(w: Workload) -> torch.Tensor:
+    """fp32 [H, D]: one seeded unit direction per head (the needles' common direction)."""
+    g = torch.Generator().manual_seed(frame_seed(w.seed, 999_983))
+    u = torch.randn((w.num_heads, w.head_dim), generator=g, dtype=torch.float32)
+    return u / u.norm(dim=1, keepdim=True)
+
+
 def draw_frame(w: Workload, t: int):
     """bf16 (q, k, v), each [T, H, D], for frame t of workload w (CPU tensors)."""
     slot = t % w.ring
@@ -137,8 +155,14 @@ def draw_frame(w: Workload, t: int):
     out = []
     for _ in range(3):
         x = torch.randn(shape, generator=g, dtype=torch.float32)
-        out.append((x * w.value_scale).to(torch.bfloat16))
-    return tuple(out)
+        out.append(x * w.value_scale)
+    if w.needle_every > 0:
+        u = needle_directions(w)
+        out[0] = out[0] + w.needle_q_gain * u[None]
+        if slot % w.needle_every == w.needle_slot:
+            out[1][0] = w.needle_k_gain * u
+            out[1][-1] = w.needle_k_gain * u
+    return tuple(x.to(torch.bfloat16) for x in out)
 
 
 def draw_ring(w: Workload, slots: int | None = None):

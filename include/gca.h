@@ -108,12 +108,25 @@ typedef struct {
   int64_t frame_idx;
   int64_t visible_keys;  /* Nk(t): keys the frame's queries see */
   int32_t logical_pages; /* pages walked, incl. partially filled ones */
-  int32_t kv_tiles;      /* 128-key tiles per query tile */
+  int32_t kv_tiles;      /* 96-key tiles per query tile */
   int32_t query_tiles;   /* 128-query tiles per head */
   int32_t grid;          /* CTAs of the attention kernel */
   int32_t split;         /* 1 if any (head, query tile) was split across CTAs (combine ran) */
   int32_t launches;      /* kernels enqueued by the call */
 } gca_attend_info;
+
+/* Counts of the attention kernels' data-dependent branches since create / the last gca_reset
+ * (all attention and combine launches of the cache). A "row" is one query row of one head. */
+typedef struct {
+  uint64_t exact_max_rows;  /* (row, key tile) pairs past a work piece's first tile whose exact
+                             * row max was computed: the bound |q| max|k| did not rule out a
+                             * rescale */
+  uint64_t rescaled_rows;   /* (row, key tile) pairs where the running max grew by more than
+                             * 2^8 and O was rescaled in tensor memory */
+  uint64_t wide_merge_rows; /* rows the split-KV combine merged from pieces whose row maxima lie
+                             * more than 2^8 apart */
+  uint64_t reserved;
+} gca_attend_counters;
 
 /* Validates a config. Host only. Returns GCA_OK, GCA_ERR_INVALID_ARG or GCA_ERR_UNSUPPORTED. */
 gca_status gca_validate_config(const gca_config* cfg);
@@ -219,7 +232,8 @@ gca_status gca_attend_prefill(gca_cache* cache, int32_t n, const void* q_rot, vo
  * It allocates nothing. Its scratch -- the split-KV partial records -- lives in a 16 MiB array
  * inside this library, which every GPU that loads the library holds until the process exits.
  * The first call on a device looks up that array's device address (cudaGetSymbolAddress) with
- * the device current; make that first call before any stream capture. The address is kept with
+ * the device current; under CUDA's lazy module loading that is also when the device commits the
+ * array's 16 MiB. Make that first call before any stream capture; later calls allocate nothing. The address is kept with
  * the CUDA context it was taken in and looked up again when the context changes (for example
  * after a cudaDeviceReset). All calls share the one
  * array and it keeps the last call's contents (every slot read is written earlier in the same
@@ -243,6 +257,26 @@ gca_status gca_cache_destroy(gca_cache* cache);
  * does nothing (its output is left unwritten) until gca_reset; appends keep running, every
  * page id range-checked before any write, so the pools stay in bounds. */
 gca_status gca_check(gca_cache* cache);
+
+/* Synchronises the device and reads the cache's attention branch counters (for tests and
+ * measurement: they show which paths of the online softmax a stream exercised). */
+gca_status gca_read_attend_counters(gca_cache* cache, gca_attend_counters* counters);
+
+/* Bound of every pipeline wait inside this cache's attention kernels, in nanoseconds (0 restores
+ * the default, 2 s). A wait that runs out -- which only a stalled pipeline can cause -- sets
+ * GCA_DEVERR_WAIT_TIMEOUT in the sticky device error word; the kernel's CTAs then stop issuing
+ * work, wait (bounded) for the copies and MMAs they already issued, free their tensor memory and
+ * return, so the call always ends and the CUDA context stays usable. Host only; applies to
+ * attention launches enqueued after the call. */
+gca_status gca_set_wait_limit(gca_cache* cache, uint64_t wait_ns);
+
+/* Test hook of the timeout path above. Arms the next attention launch of this cache
+ * (gca_attend, gca_attend_prefill or gca_attend_noalloc): in it, CTA 0 never issues the copies
+ * of its first key tile (nothing is ever in flight for that tile), so its MMA issuer's wait for
+ * them runs out after the wait limit and the launch sets GCA_DEVERR_WAIT_TIMEOUT. The combine
+ * launch of the call then does nothing (sticky error), so no output row that depends on a
+ * split work unit is written; gca_check reports GCA_ERR_DEVICE until gca_reset. One-shot. */
+gca_status gca_test_withhold_copies(gca_cache* cache);
 
 /* Fills *state from the host mirror (no GPU access). */
 gca_status gca_get_state(const gca_cache* cache, gca_state* state);

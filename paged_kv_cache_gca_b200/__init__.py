@@ -20,6 +20,8 @@ __all__ = [
     "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc", "gca_append_frames",
     "gca_append_frame_ex", "gca_rollback_last_frame", "gca_attend_prefill",
     "GCA_APPEND_TRANSIENT", "GcaCache", "config_for", "EXPORTED_SYMBOLS",
+    "gca_set_wait_limit", "gca_test_withhold_copies", "gca_read_attend_counters",
+    "GcaAttendCounters",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -76,12 +78,20 @@ class GcaAttendInfo(ctypes.Structure):
     ]
 
 
+class GcaAttendCounters(ctypes.Structure):
+    _fields_ = [
+        ("exact_max_rows", ctypes.c_uint64), ("rescaled_rows", ctypes.c_uint64),
+        ("wide_merge_rows", ctypes.c_uint64), ("reserved", ctypes.c_uint64),
+    ]
+
+
 # Every symbol include/gca.h declares.
 EXPORTED_SYMBOLS = (
     "gca_validate_config", "gca_workspace_bytes", "gca_cache_create", "gca_append_frame",
     "gca_attend", "gca_reset", "gca_cache_destroy", "gca_check", "gca_get_state",
     "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc", "gca_append_frames",
     "gca_append_frame_ex", "gca_rollback_last_frame", "gca_attend_prefill",
+    "gca_set_wait_limit", "gca_test_withhold_copies", "gca_read_attend_counters",
 )
 
 _lib = None
@@ -116,6 +126,9 @@ def lib():
         "gca_append_frame_ex": (I32, [VP, I64, I64, ctypes.c_uint32, VP, VP, VP, VP, VP]),
         "gca_rollback_last_frame": (I32, [VP, I64, VP]),
         "gca_attend_prefill": (I32, [VP, I32, VP, VP, VP]),
+        "gca_set_wait_limit": (I32, [VP, ctypes.c_uint64]),
+        "gca_test_withhold_copies": (I32, [VP]),
+        "gca_read_attend_counters": (I32, [VP, P(GcaAttendCounters)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -187,6 +200,21 @@ def gca_append_frames(handles, frame_idx, q_ptrs, k_ptrs, v_ptrs, q_rot_ptrs, st
     _ok(lib().gca_append_frames(arr(VP, handles), n, arr(I64, frame_idx), arr(VP, q_ptrs),
                                 arr(VP, k_ptrs), arr(VP, v_ptrs), arr(VP, q_rot_ptrs), stream),
         "gca_append_frames")
+
+
+def gca_set_wait_limit(handle, wait_ns: int) -> None:
+    _ok(lib().gca_set_wait_limit(handle, wait_ns), "gca_set_wait_limit")
+
+
+def gca_test_withhold_copies(handle) -> None:
+    """Test hook: the next attention launch's CTA 0 never issues its first tile's copies."""
+    _ok(lib().gca_test_withhold_copies(handle), "gca_test_withhold_copies")
+
+
+def gca_read_attend_counters(handle) -> GcaAttendCounters:
+    out = GcaAttendCounters()
+    _ok(lib().gca_read_attend_counters(handle, ctypes.byref(out)), "gca_read_attend_counters")
+    return out
 
 
 def gca_reset(handle, stream) -> None:
@@ -299,6 +327,10 @@ class GcaCache:
 
     def attend_info(self) -> GcaAttendInfo:
         return gca_last_attend_info(self.handle)
+
+    def counters(self) -> GcaAttendCounters:
+        """Attention branch counters since create / reset (synchronises)."""
+        return gca_read_attend_counters(self.handle)
 
     def _view(self, ptr, count, dtype):
         import torch

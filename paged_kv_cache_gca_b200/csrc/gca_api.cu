@@ -3,9 +3,11 @@
 // the caller's workspace; the host handle holds only counters that evolve deterministically,
 // so no call needs to read anything back from the GPU (only gca_check does).
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -13,6 +15,16 @@
 #include "gca_internal.h"
 
 namespace gca {
+
+bool nvtx_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("GCA_NVTX");
+    return e != nullptr && e[0] == '1';
+  }();
+  return on;
+}
+void nvtx_push(const char* name) { nvtxRangePushA(name); }
+void nvtx_pop() { nvtxRangePop(); }
 
 namespace {
 
@@ -136,6 +148,7 @@ bool compute_layout(const gca_config& c, Layout* L) {
   L->rope_tok = take(8 * (size_t)T * (L->ny + L->nx));
   L->err = take(4);
   L->kmax = take(4 * (size_t)c.num_heads);
+  L->counters = take(8 * 4);
   L->part_o = take(4 * (size_t)L->part_slots * kTileQ * kHeadDim);
   L->part_ml = take(8 * (size_t)L->part_slots * kTileQ);
   L->total = align_up(off, kAlign);
@@ -163,6 +176,7 @@ bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams
   p->traj_pages = reinterpret_cast<const int32_t*>(c->ws + L.traj_pages);
   p->err = reinterpret_cast<uint32_t*>(c->ws + L.err);
   p->kmax = reinterpret_cast<const uint32_t*>(c->ws + L.kmax);
+  p->counters = reinterpret_cast<unsigned long long*>(c->ws + L.counters);
   if (q_rows <= 0) q_rows = L.T;
   const int32_t n_qt = (int32_t)((q_rows + kTileQ - 1) / kTileQ);
   p->T = (int32_t)q_rows;
@@ -192,6 +206,8 @@ bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams
   g = std::min<int64_t>(g, p->total);
   p->grid = (int32_t)g;
   p->scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)cf.head_dim));
+  p->wait_ns = c->wait_ns > 0 ? c->wait_ns : kDefaultWaitNs;
+  p->withhold = c->withhold_next;
   bool sp = false;
   for (int u = 0; u < p->units2 && !sp; ++u) {
     const int64_t first = (int64_t)u * p->n_tiles;
@@ -259,6 +275,7 @@ size_t gca_workspace_bytes(const gca_config* cfg) {
 gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t ws_bytes,
                             const int32_t* dev_initial_free_list, void* stream,
                             gca_cache** out) {
+  NvtxRange range_("gca_cache_create");
   if (!out) return GCA_ERR_INVALID_ARG;
   *out = nullptr;
   gca_status st = validate(cfg);
@@ -309,7 +326,8 @@ gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t w
                 cudaSuccess &&
             cudaMemsetAsync(c->ws + L.seen, 0, 4 * (size_t)cfg->num_pages, s) == cudaSuccess &&
             cudaMemsetAsync(c->ws + L.err, 0, 4, s) == cudaSuccess &&
-            cudaMemsetAsync(c->ws + L.kmax, 0, 4 * (size_t)cfg->num_heads, s) == cudaSuccess;
+            cudaMemsetAsync(c->ws + L.kmax, 0, 4 * (size_t)cfg->num_heads, s) == cudaSuccess &&
+            cudaMemsetAsync(c->ws + L.counters, 0, 8 * 4, s) == cudaSuccess;
   if (ok) {
     InitParams ip;
     std::memset(&ip, 0, sizeof(ip));
@@ -341,6 +359,7 @@ gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t w
     return GCA_ERR_CUDA;
   }
   c->free_tail = cfg->num_pages;
+  c->wait_ns = kDefaultWaitNs;
   *out = c;
   return GCA_OK;
 }
@@ -446,6 +465,7 @@ void commit_append(gca_cache* c, const AppendParams& p, bool transient) {
 gca_status gca_append_frame_ex(gca_cache* c, int64_t t, int64_t rope_frame, uint32_t flags,
                                const void* q, const void* k, const void* v, void* q_rot_out,
                                void* stream) {
+  NvtxRange range_("gca_append_frame_ex");
   AppendParams p;
   const gca_status st = prepare_append(c, t, rope_frame, flags, q, k, v, q_rot_out, &p);
   if (st != GCA_OK) return st;
@@ -460,6 +480,7 @@ gca_status gca_append_frame(gca_cache* c, int64_t t, const void* q, const void* 
 }
 
 gca_status gca_rollback_last_frame(gca_cache* c, int64_t t, void* /*stream*/) {
+  NvtxRange range_("gca_rollback_last_frame");
   if (!c) return GCA_ERR_INVALID_ARG;
   if (!c->transient || c->frames == 0 || t != c->frames - 1) return GCA_ERR_FRAME_ORDER;
   // A transient append popped exactly ppf pages from the head and pushed none; moving the
@@ -473,6 +494,7 @@ gca_status gca_rollback_last_frame(gca_cache* c, int64_t t, void* /*stream*/) {
 gca_status gca_append_frames(gca_cache* const* caches, int32_t n, const int64_t* frame_idx,
                              const void* const* q, const void* const* k, const void* const* v,
                              void* const* q_rot_out, void* stream) {
+  NvtxRange range_("gca_append_frames");
   if (!caches || !frame_idx || !q || !k || !v || !q_rot_out) return GCA_ERR_INVALID_ARG;
   if (n < 1 || n > kMaxAppendBatch) return GCA_ERR_INVALID_ARG;
   static thread_local AppendBatch b;  // ~30 KB: kept off the stack
@@ -517,6 +539,7 @@ gca_status enqueue_attention(gca_cache* c, int64_t t, int64_t q_rows, const void
   p.part_ml = at<float2>(c, L.part_ml);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (launch_attn(c->tm_k, c->tm_v, p, s) != cudaSuccess) return GCA_ERR_CUDA;
+  c->withhold_next = 0;
   if (split && launch_combine(p, s) != cudaSuccess) return GCA_ERR_CUDA;
 
   gca_attend_info& inf = c->last;
@@ -534,6 +557,7 @@ gca_status enqueue_attention(gca_cache* c, int64_t t, int64_t q_rows, const void
 }  // namespace
 
 gca_status gca_attend(gca_cache* c, int64_t t, const void* q_rot, void* out, void* stream) {
+  NvtxRange range_("gca_attend");
   if (!c || !q_rot || !out || !aligned16(q_rot) || !aligned16(out)) return GCA_ERR_INVALID_ARG;
   if (c->frames == 0 || t != c->frames - 1) return GCA_ERR_FRAME_ORDER;
   if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;
@@ -544,6 +568,7 @@ gca_status gca_attend(gca_cache* c, int64_t t, const void* q_rot, void* out, voi
 
 gca_status gca_attend_prefill(gca_cache* c, int32_t n, const void* q_rot, void* out,
                               void* stream) {
+  NvtxRange range_("gca_attend_prefill");
   if (!c || !q_rot || !out || !aligned16(q_rot) || !aligned16(out)) return GCA_ERR_INVALID_ARG;
   if (n < 1 || n > c->cfg.anchor_frames) return GCA_ERR_INVALID_ARG;
   if (c->frames != n || c->transient) return GCA_ERR_FRAME_ORDER;
@@ -555,6 +580,7 @@ gca_status gca_attend_prefill(gca_cache* c, int32_t n, const void* q_rot, void* 
 }
 
 gca_status gca_reset(gca_cache* c, void* stream) {
+  NvtxRange range_("gca_reset");
   if (!c) return GCA_ERR_INVALID_ARG;
   if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;
   const Layout& L = c->lay;
@@ -562,7 +588,9 @@ gca_status gca_reset(gca_cache* c, void* stream) {
                    at<uint32_t>(c, L.err), c->cfg.num_pages,
                    static_cast<cudaStream_t>(stream)) != cudaSuccess ||
       cudaMemsetAsync(c->ws + L.kmax, 0, 4 * (size_t)c->cfg.num_heads,
-                      static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess ||
+      cudaMemsetAsync(c->ws + L.counters, 0, 8 * 4, static_cast<cudaStream_t>(stream)) !=
+          cudaSuccess) {
     return GCA_ERR_CUDA;
   }
   c->frames = 0;
@@ -582,6 +610,7 @@ gca_status gca_cache_destroy(gca_cache* c) {
 }
 
 gca_status gca_check(gca_cache* c) {
+  NvtxRange range_("gca_check");
   if (!c) return GCA_ERR_INVALID_ARG;
   if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return GCA_ERR_CUDA;
@@ -614,6 +643,34 @@ gca_status gca_get_state(const gca_cache* c, gca_state* s) {
   s->traj_page_list = reinterpret_cast<int32_t*>(c->ws + L.traj_pages);
   s->slot_map = reinterpret_cast<int32_t*>(c->ws + L.slot_map);
   s->kept_tokens = reinterpret_cast<int32_t*>(c->ws + L.kept);
+  return GCA_OK;
+}
+
+gca_status gca_read_attend_counters(gca_cache* c, gca_attend_counters* out) {
+  NvtxRange range_("gca_read_attend_counters");
+  if (!c || !out) return GCA_ERR_INVALID_ARG;
+  if (!on_cache_device(c)) return GCA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return GCA_ERR_CUDA;
+  uint64_t v[4] = {0, 0, 0, 0};
+  if (cudaMemcpy(v, c->ws + c->lay.counters, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    return GCA_ERR_CUDA;
+  }
+  std::memset(out, 0, sizeof(*out));
+  out->exact_max_rows = v[0];
+  out->rescaled_rows = v[1];
+  out->wide_merge_rows = v[2];
+  return GCA_OK;
+}
+
+gca_status gca_set_wait_limit(gca_cache* c, uint64_t wait_ns) {
+  if (!c) return GCA_ERR_INVALID_ARG;
+  c->wait_ns = wait_ns > 0 ? wait_ns : kDefaultWaitNs;
+  return GCA_OK;
+}
+
+gca_status gca_test_withhold_copies(gca_cache* c) {
+  if (!c) return GCA_ERR_INVALID_ARG;
+  c->withhold_next = 1;
   return GCA_OK;
 }
 

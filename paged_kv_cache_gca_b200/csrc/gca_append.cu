@@ -271,18 +271,16 @@ __device__ __forceinline__ void append_block(const AppendParams& p, const int bx
 #define GCA_APPEND_BOUNDS __launch_bounds__(512, 4)
 
 __global__ void GCA_APPEND_BOUNDS append_kernel(const AppendParams p) {
-  pdl_signal_early();
   pdl_wait();  // inputs, pages and the free ring may come from earlier work in the stream
   append_block(p, (int)blockIdx.x);
-  pdl_signal_late();
+  pdl_launch_dependents();
 }
 
 __global__ void GCA_APPEND_BOUNDS append_batch_kernel(const __grid_constant__ AppendBatch b) {
-  pdl_signal_early();
   pdl_wait();
   const AppendParams& p = b.p[blockIdx.y];
   if ((int)blockIdx.x < p.n_blocks) append_block(p, (int)blockIdx.x);
-  pdl_signal_late();
+  pdl_launch_dependents();
 }
 
 }  // namespace

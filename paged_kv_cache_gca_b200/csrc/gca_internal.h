@@ -20,10 +20,12 @@ constexpr int kPageSize = 16;
 constexpr int kMaxHeads = 64;
 constexpr int kMaxKeep = 64;
 constexpr int kTileQ = 128;     // query rows per attention tile
-constexpr int kTileK = 128;     // keys per attention tile (8 pages)
+constexpr int kTileK = 96;      // keys per attention tile (6 pages): two S/P buffers of 96
+                                // columns and O (64) per query tile fill 256 TMEM columns
 constexpr int kQPerCta = 2;     // query tiles per attention CTA: a work unit is a pair of tiles
                                 // of one head (they share every K/V tile)
 constexpr int kPagesPerTile = kTileK / kPageSize;
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // bound of every attention pipeline wait
 constexpr int kMaxGrid = 512;   // attention CTAs per launch (sizes the split buffers)
 constexpr size_t kAlign = 1024;
 constexpr int kMaxAppendBatch = 128;  // caches per batched append launch (kernel-parameter bound)
@@ -31,34 +33,12 @@ constexpr int kMaxAppendBatch = 128;  // caches per batched append launch (kerne
 // Programmatic dependent launch: the append, attention and combine kernels are launched with
 // programmatic stream serialization, signal their dependents once their main work is done and
 // wait for their prerequisites (griddepcontrol.wait) before touching any data that earlier work
-// in the stream produced, so a kernel's launch overlaps the previous kernel's tail. Signalling
-// at the start instead lets the next grids' blocks take SMs early and wait there (slower). A
+// in the stream produced, so a kernel's launch overlaps the previous kernel's tail. A
 // prerequisite that never signals (any kernel outside this library) is waited for to its end.
-#ifndef GCA_PDL
-#define GCA_PDL 1
-#endif
-// GCA_PDL_LATE 1: kernels signal their dependents after their main work; 0: at their start.
-#ifndef GCA_PDL_LATE
-#define GCA_PDL_LATE 1
-#endif
-
 #ifdef __CUDACC__
-__device__ __forceinline__ void pdl_wait() {
-#if GCA_PDL
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-#endif
-}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
-#if GCA_PDL
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-#endif
-}
-// Signal points at the start and at the end of a kernel's main work; one of them is active.
-__device__ __forceinline__ void pdl_signal_early() {
-  if (!GCA_PDL_LATE) pdl_launch_dependents();
-}
-__device__ __forceinline__ void pdl_signal_late() {
-  if (GCA_PDL_LATE) pdl_launch_dependents();
 }
 
 // Launches kernel<<<grid, block, smem, s>>>(args...) with programmatic stream serialization.
@@ -72,12 +52,27 @@ inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 bl
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = GCA_PDL ? 1 : 0;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 #endif
+
+// NVTX ranges around the C-ABI entry points, for timeline profilers: off unless the process
+// runs with GCA_NVTX=1 (read once). With no profiler attached a range costs a function call.
+bool nvtx_enabled();
+void nvtx_push(const char* name);
+void nvtx_pop();
+struct NvtxRange {
+  bool on;
+  explicit NvtxRange(const char* name) : on(nvtx_enabled()) {
+    if (on) nvtx_push(name);
+  }
+  ~NvtxRange() {
+    if (on) nvtx_pop();
+  }
+};
 
 // Byte offsets of every region inside the caller's workspace.
 struct Layout {
@@ -93,6 +88,7 @@ struct Layout {
   size_t rope_tok;           // float2 (cos, sin) [T][ny + nx]: spatial bands per token
   size_t err;                // uint32 sticky device error word
   size_t kmax;               // float [H] (as uint32 bits): max squared key norm ever appended
+  size_t counters;           // uint64 [4]: attention branch counters (gca_read_attend_counters)
   size_t part_o;             // float [part_slots][128][64]
   size_t part_ml;            // float2 [part_slots][128]
   size_t total;
@@ -178,6 +174,8 @@ struct AttnParams {
   const int32_t* traj_pages;
   uint32_t* err;
   const uint32_t* kmax;  // per head: max squared key norm of everything appended
+  unsigned long long* counters;  // [0] exact row max after a segment's first tile, [1] O
+                                 // rescales, [2] rows merged over maxima more than 2^8 apart
   int32_t T;  // query rows of the launch (T of one frame, or n * T for a joint prefill)
   int32_t H, ppf, last_len, num_pages;
   int32_t na_pages;      // anchor pages (visible anchor frames * ppf)
@@ -186,7 +184,7 @@ struct AttnParams {
   int32_t n_traj_pages;
   int32_t traj_tail_len; // valid slots of the last trajectory page
   int32_t n_lp;          // logical pages walked
-  int32_t n_tiles;       // 128-key tiles
+  int32_t n_tiles;       // key tiles of kTileK keys
   int32_t n_qt;          // 128-query tiles per head
   int32_t units;         // H * n_qt: (head, query tile) pairs, the combine grid
   int32_t n_pairs;       // query-tile pairs per head (a CTA works on two tiles of one head)
@@ -194,6 +192,9 @@ struct AttnParams {
   int64_t total;         // units2 * n_tiles
   int32_t grid;
   float scale_log2;      // log2(e) / sqrt(D)
+  uint64_t wait_ns;      // bound of every pipeline wait (a wait that runs out sets
+                         // GCA_DEVERR_WAIT_TIMEOUT and the CTA winds down)
+  int32_t withhold;      // test hook: 1 = CTA 0 never issues the copies of its first key tile
 };
 
 // Launchers (return cudaGetLastError() of the launch).
@@ -245,6 +246,8 @@ struct gca_cache {
   int32_t n_kept;
   int32_t kept[gca::kMaxKeep];
   uint32_t dev_err;
+  uint64_t wait_ns;        // attention wait bound (gca_set_wait_limit)
+  int32_t withhold_next;   // test hook armed for the next attention launch
   CUtensorMap tm_k;
   CUtensorMap tm_v;
   gca_attend_info last;

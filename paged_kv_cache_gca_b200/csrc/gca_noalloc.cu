@@ -87,6 +87,7 @@ using namespace gca;
 
 extern "C" gca_status gca_attend_noalloc(gca_cache* c, int64_t t, const void* q_rot, void* out,
                                          void* stream) {
+  NvtxRange range_("gca_attend_noalloc");
   if (!c || !q_rot || !out) return GCA_ERR_INVALID_ARG;
   // 16-byte vector accesses: a misaligned tensor is rejected here, not faulted on the device
   if (((reinterpret_cast<uintptr_t>(q_rot) | reinterpret_cast<uintptr_t>(out)) & 15u) != 0) {
@@ -114,6 +115,7 @@ extern "C" gca_status gca_attend_noalloc(gca_cache* c, int64_t t, const void* q_
                                         (size_t)kNoallocSlots * kSlotOBytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (launch_attn(c->tm_k, c->tm_v, p, s) != cudaSuccess) return GCA_ERR_CUDA;
+  c->withhold_next = 0;
   if (split && launch_combine(p, s) != cudaSuccess) return GCA_ERR_CUDA;
   return GCA_OK;
 }
