@@ -29,6 +29,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import gca_inputs as gi  # noqa: E402
+import paged_kv_cache_gca_b200 as gca  # noqa: E402
+from paged_kv_cache_gca_b200 import build as gbuild  # noqa: E402
 
 METRIC = "GCA frames/sec and attention TFLOP/s (% of BF16 peak) at 1 B200"
 WORKLOAD = "w16_320"
@@ -155,10 +157,67 @@ def traffic_from_profile(kernel: str):
     return ent.get("dram_bytes_per_launch")
 
 
-def run_ours(args, rank, world, device):
-    import paged_kv_cache_gca_b200 as gca
-    from paged_kv_cache_gca_b200 import build as gbuild
+def attn_flops(w: gi.Workload, visible: int) -> float:
+    """Algorithmic attention work of one frame: QK^T and PV over the visible keys only."""
+    return 4.0 * w.num_heads * w.head_dim * w.tokens_per_frame * visible
 
+
+def stream_frames(cache, ring, w, stream, q_rot, out, frames, ev=None, reattend=False,
+                  flops=None):
+    """Appends and attends frames of w from the device ring (one cache). ev[t]: 4 events
+    (before the append, after it, between the attention and combine launches, after the call).
+    reattend: every frame's attention is run a second time (it reads the same state, so the
+    difference to a plain pass is the attention's own time)."""
+    for t in frames:
+        q, k, v = ring[t % w.ring]
+        if ev is not None:
+            ev[t][0].record(stream)
+            gca.gca_set_split_event(cache.handle, ev[t][2].cuda_event)
+        cache.append_frame(t, q, k, v, q_rot, stream=stream)
+        if ev is not None:
+            ev[t][1].record(stream)
+        cache.attend(t, q_rot, out, stream=stream)
+        if ev is not None:
+            ev[t][3].record(stream)
+        if reattend:
+            cache.attend(t, q_rot, out, stream=stream)
+        if flops is not None and len(flops) < len(frames):
+            flops.append(attn_flops(w, cache.attend_info().visible_keys))
+    if ev is not None:
+        gca.gca_set_split_event(cache.handle, None)
+
+
+def new_events(n):
+    """n groups of 4 timing events, each recorded once so that its CUDA handle exists."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+    for g in evs:
+        for e in g:
+            e.record()
+    torch.cuda.synchronize()
+    return evs
+
+
+def split_times(ev, frames):
+    """(append ms, attention kernel ms, combine ms) summed over the frames."""
+    a = sum(ev[t][0].elapsed_time(ev[t][1]) for t in frames)
+    k = sum(ev[t][1].elapsed_time(ev[t][2]) for t in frames)
+    c = sum(ev[t][2].elapsed_time(ev[t][3]) for t in frames)
+    return a, k, c
+
+
+def timed(stream, fn):
+    """Device time (ms) of the work fn enqueues on stream, synchronised on both sides."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def run_ours(args, rank, world, device):
     gbuild.build()
     w = gi.workload(args.workload)
     T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
@@ -171,41 +230,35 @@ def run_ours(args, rank, world, device):
     q_rot = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
     out = torch.empty_like(q_rot)
     nframes = w.frames
-
-    # per-frame work (host values the library reports)
+    frames = range(nframes)
     flops = []
-    info_launches = []
 
-    def one_step(events=None):
+    def one_step(ev=None, reattend=False):
         cache.reset(stream=stream)
-        for t in range(nframes):
-            q, k, v = ring[t % w.ring]
-            if events is not None:
-                events[t][0].record(stream)
-            cache.append_frame(t, q, k, v, q_rot, stream=stream)
-            if events is not None:
-                events[t][1].record(stream)
-            cache.attend(t, q_rot, out, stream=stream)
-            if events is not None:
-                events[t][2].record(stream)
-            if len(flops) < nframes:
-                inf = cache.attend_info()
-                flops.append(4.0 * H * D * T * inf.visible_keys)
-                info_launches.append(inf.launches)
+        stream_frames(cache, ring, w, stream, q_rot, out, frames, ev=ev, reattend=reattend,
+                      flops=flops)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             one_step()
     torch.cuda.synchronize(device)
     assert cache.check() == 0, "device error after warm-up"
+    # kernels per frame: append + attention (+ combine when the key range is split)
+    per_frame_launches = []
+    with torch.cuda.stream(stream):
+        cache.reset(stream=stream)
+        for t in frames:
+            q, k, v = ring[t % w.ring]
+            cache.append_frame(t, q, k, v, q_rot, stream=stream)
+            cache.attend(t, q_rot, out, stream=stream)
+            per_frame_launches.append(1 + cache.attend_info().launches)
+    torch.cuda.synchronize(device)
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
-    # one event triple per (step, frame): read only after the timed region
-    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nframes)]
-          for _ in range(args.steps)]
+    ev = [new_events(nframes) for _ in range(args.steps)]
     e_start = torch.cuda.Event(enable_timing=True)
     e_stop = torch.cuda.Event(enable_timing=True)
     clocks_path = args.clocks_csv  # raw nvidia-smi samples, when asked for
@@ -216,57 +269,214 @@ def run_ours(args, rank, world, device):
         torch.cuda.synchronize(device)
         e_start.record(stream)
         with torch.cuda.stream(stream):
-            for s in range(args.steps):
+            for _ in range(args.steps):
                 one_step()
         e_stop.record(stream)
         torch.cuda.synchronize(device)
         barrier()
-        # the per-call breakdown: the same K steps with events around every call (an event
+        # per-kernel breakdown: the same K steps with events around every launch (an event
         # between two kernels also stops the next launch from overlapping the previous tail)
         with torch.cuda.stream(stream):
             for s in range(args.steps):
                 one_step(ev[s])
         torch.cuda.synchronize(device)
-    append_ms = sum(e[0].elapsed_time(e[1]) for st in ev for e in st)
-    attend_ms = sum(e[1].elapsed_time(e[2]) for st in ev for e in st)
+        # exposed append: a plain pass that attends every frame twice; the second attention
+        # reads the same state, so (twice the plain step - this step) is the time the append
+        # adds to a frame
+        re_ms = timed(stream, lambda: [one_step(reattend=True) for _ in range(args.steps)])
     elapsed_ms = e_start.elapsed_time(e_stop)
+    app_ms = attn_ms = comb_ms = 0.0
+    for s in range(args.steps):
+        a, k, c = split_times(ev[s], frames)
+        app_ms, attn_ms, comb_ms = app_ms + a, attn_ms + k, comb_ms + c
     assert cache.check() == 0, "device error in the timed region"
-    step_ms_calls = (append_ms + attend_ms) / args.steps
-
     elapsed_ms = max_over_ranks(elapsed_ms, world, device)
 
     # ---- end-to-end through the public API with host buffers (pinned), copies timed
     e2e = run_e2e(args, w, cache, ring_host, device, stream, world)
-    batched = run_batched_append(ring, device, stream) if world == 1 else None
-    prefill = run_prefill(ring, device, stream) if world == 1 else None
-    keyframes = run_keyframe_stream(ring, device, stream) if world == 1 else None
-    camera = run_camera_head(device, stream) if world == 1 else None
-    windowed_mode = run_windowed(ring, device, stream) if world == 1 else None
+    extra = {}
+    if world == 1:
+        extra["batched"] = run_batched_append(ring, device, stream)
+        extra["prefill"] = run_prefill(ring, device, stream)
+        extra["keyframes"] = run_keyframe_stream(ring, device, stream)
+        extra["camera"] = run_camera_head(device, stream)
+        extra["windowed"] = run_windowed(ring, device, stream)
+        if not args.main_only:
+            extra["configs"] = run_configs(args, device, stream)
 
     res = {
         "elapsed_ms": elapsed_ms,
-        "step_ms_calls": step_ms_calls,
-        "attend_ms_per_step": attend_ms / args.steps,
-        "append_ms_per_step": append_ms / args.steps,
-        "flops_per_step": float(sum(flops)),
-        "launches_per_step": 1 + nframes + int(sum(info_launches)),
+        "attn_ms_per_step": attn_ms / args.steps,
+        "combine_ms_per_step": comb_ms / args.steps,
+        "append_ms_per_step": app_ms / args.steps,
+        "reattend_ms_per_step": re_ms / args.steps,
+        "flops_per_step": float(sum(flops[:nframes])),
+        "launches_per_step": 1 + int(sum(per_frame_launches)),
         "clocks": clk.summary(),
         "e2e": e2e,
         "frames": nframes,
-        "batched_append": batched,
-        "prefill": prefill,
-        "keyframes": keyframes,
-        "camera": camera,
-        "windowed": windowed_mode,
+        **extra,
     }
     cache.close()
     return w, res
 
 
+def run_stream_config(w, device, stream, warm=1, timed_passes=1, span=None, events=True):
+    """frames/s of one cache streaming workload w (device ring inputs), attention TFLOP/s of the
+    stream and of the attention kernel alone (an instrumented pass with events around each
+    launch). span: the frames timed (a contiguous range ending at the last frame); the frames
+    before it are streamed untimed first."""
+    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    ring = gi.draw_ring(w).to(device)
+    with torch.cuda.stream(stream):
+        cache = gca.GcaCache(gca.config_for(w), initial_free=gi.initial_free_list(w),
+                             stream=stream)
+    q_rot = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
+    out = torch.empty_like(q_rot)
+    first = 0 if span is None else w.frames - span
+    head, body = range(first), range(first, w.frames)
+    flops = []
+
+    def prefix():
+        cache.reset(stream=stream)
+        stream_frames(cache, ring, w, stream, q_rot, out, head)
+
+    def body_pass(ev=None, fl=None):
+        stream_frames(cache, ring, w, stream, q_rot, out, body, ev=ev, flops=fl)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            prefix()
+            body_pass(fl=flops)
+    ms = 0.0
+    for _ in range(timed_passes):
+        with torch.cuda.stream(stream):
+            prefix()
+        ms += timed(stream, body_pass)
+    ms /= timed_passes
+    res = {"frames_timed": len(body), "first_frame_timed": first,
+           "frames_per_s": len(body) / (ms / 1e3), "ms": ms,
+           "attention_tflops_stream": sum(flops) / (ms / 1e3) / 1e12}
+    if events:
+        ev = new_events(w.frames)
+        with torch.cuda.stream(stream):
+            prefix()
+            body_pass(ev=ev)
+        torch.cuda.synchronize()
+        a, k, c = split_times(ev, body)
+        res.update({"attn_kernel_tflops": sum(flops) / (k / 1e3) / 1e12,
+                    "attn_kernel_us_per_frame": 1e3 * k / len(body),
+                    "combine_us_per_frame": 1e3 * c / len(body),
+                    "append_us_per_frame": 1e3 * a / len(body)})
+    assert cache.check() == 0, f"device error in {w.name}"
+    cnt = cache.counters()
+    res["branch_counters"] = {"exact_max_rows": cnt.exact_max_rows,
+                              "rescaled_rows": cnt.rescaled_rows,
+                              "wide_merge_rows": cnt.wide_merge_rows}
+    cache.close()
+    return res
+
+
+def run_stack(device, warm=1):
+    """stack24x4: 24 layer caches on each of 4 concurrent streams (4 CUDA streams), 500 frames;
+    per stream and frame one gca_append_frames over its 24 caches, then 24 attentions."""
+    w = gi.workload("stack24x4")
+    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
+    ring = gi.draw_ring(w).to(device)
+    R = ring.shape[0]
+    streams = [torch.cuda.Stream(device=device) for _ in range(w.num_streams)]
+    caches = {}
+    for s in range(w.num_streams):
+        with torch.cuda.stream(streams[s]):
+            for layer in range(w.num_layers):
+                caches[s, layer] = gca.GcaCache(
+                    gca.config_for(w, gi.rope_base_for_layer(w, layer)), stream=streams[s])
+    q_rot = {k: torch.empty((T, H, D), dtype=torch.bfloat16, device=device) for k in caches}
+    out = {k: torch.empty((T, H, D), dtype=torch.bfloat16, device=device) for k in caches}
+    fb = T * H * D * 2
+    base = ring.data_ptr()
+    flops = [0.0]
+
+    def one_pass(count):
+        for s in range(w.num_streams):
+            for layer in range(w.num_layers):
+                caches[s, layer].reset(stream=streams[s])
+        for t in range(w.frames):
+            for s in range(w.num_streams):
+                slot = (4 * t + s) % R
+                ptr = [base + (3 * slot + j) * fb for j in range(3)]
+                keys = [(s, layer) for layer in range(w.num_layers)]
+                gca.gca_append_frames([caches[k].handle for k in keys], [t] * len(keys),
+                                      [ptr[0]] * len(keys), [ptr[1]] * len(keys),
+                                      [ptr[2]] * len(keys), [q_rot[k].data_ptr() for k in keys],
+                                      streams[s].cuda_stream)
+                for k in keys:
+                    caches[k].attend(t, q_rot[k], out[k], stream=streams[s])
+                    if count:
+                        flops[0] += attn_flops(w, caches[k].attend_info().visible_keys)
+
+    for _ in range(warm):
+        one_pass(False)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(streams[0])
+    for s in streams[1:]:
+        s.wait_event(e0)
+    one_pass(True)
+    for s in streams[1:]:
+        streams[0].wait_stream(s)
+    e1.record(streams[0])
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    assert all(c.check() == 0 for c in caches.values()), "device error in the stack"
+    layer_frames = w.frames * w.num_streams * w.num_layers
+    for c in caches.values():
+        c.close()
+    return {"frames_per_s": w.frames * w.num_streams / (ms / 1e3),
+            "layer_frames_per_s": layer_frames / (ms / 1e3),
+            "us_per_layer_frame": 1e3 * ms / layer_frames, "ms": ms,
+            "attention_tflops_stream": flops[0] / (ms / 1e3) / 1e12,
+            "host_enqueue_s": round(time.perf_counter() - t0, 3)}
+
+
+def run_configs(args, device, stream):
+    """The other workloads of the pages' 518x378 layer, one line each."""
+    pk, _ = peaks()
+    burst = pk["bf16_tflops"]
+    out = {}
+    w = gi.workload("w16_320").replace(value_scale=1.0)
+    r = run_stream_config(w, device, stream, warm=1, timed_passes=2)
+    out["w16_320_unit_variance"] = {"workload": "w16_320 with q, k, v ~ N(0,1) (the row-max "
+                                                "bound no longer skips the exact max)", **r}
+    for name, span in (("w64_1000", None), ("w32_10k", None)):
+        w = gi.workload(name)
+        r = run_stream_config(w, device, stream, warm=1, timed_passes=1, span=span)
+        out[name] = {"workload": f"{name}: " + workload_desc(w), **r}
+    out["stack24x4"] = {"workload": "stack24x4: " + workload_desc(gi.workload("stack24x4")) +
+                        ", 24 layers x 4 concurrent streams", **run_stack(device)}
+    for k, v in out.items():
+        for key in ("attn_kernel_tflops", "attention_tflops_stream"):
+            if key in v:
+                v[key.replace("tflops", "frac_of_burst")] = v[key] / burst
+    if not args.no_cpu_baseline:
+        for name in ("w64_1000", "w32_10k", "stack24x4"):
+            w = gi.workload(name)
+            sample = [w.frames // 2, w.frames - 1]
+            v, d = oracle_frames_per_s(w, sample, rows=64)
+            out[name]["cpu_baseline"] = {
+                "value": v, "unit": "frames/s", "cores": blas_threads(), "kind": "oracle",
+                "sample": (f"FIFO bookkeeping over all {w.frames} frames + fp64 attention of 64 "
+                           f"random rows x all heads of frames {sample[0]} and {sample[1]}, "
+                           "extrapolated to the stream by query-key pairs"
+                           + (" (one layer of one stream)" if name == "stack24x4" else "")),
+                **d}
+    return out
+
+
 def run_prefill(ring, device, stream, warm=3, timed=10):
     """Joint bidirectional attention of the 8 scale frames (gca_attend_prefill): 8*T = 8032
     queries over 8032 keys per head, 264 GFLOP. Frames from the device ring."""
-    import paged_kv_cache_gca_b200 as gca
 
     w = gi.workload("scale8")
     n = w.anchor_frames
@@ -304,7 +514,6 @@ def run_prefill(ring, device, stream, warm=3, timed=10):
 def run_keyframe_stream(ring, device, stream, interval=5):
     """The 320-frame stream with keyframe-only caching: every 5th video frame is kept, the
     others append transiently, attend and roll back (one untimed pass, one timed pass)."""
-    import paged_kv_cache_gca_b200 as gca
 
     w = gi.workload(WORKLOAD)
     T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
@@ -354,7 +563,6 @@ def run_camera_head(device, stream):
     32 heads, window 16, K = 1. Per frame, layer by layer as a trunk runs them: append, then
     attend (one query row per head over up to 1024 keys: the decode-like regime). One untimed
     pass, one timed pass of the 1024-frame stream."""
-    import paged_kv_cache_gca_b200 as gca
 
     w = gi.workload("camera4")
     T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
@@ -397,7 +605,6 @@ def run_windowed(ring, device, stream, total=1000, window=128, overlap=8):
     """Windowed mode (--mode windowed --window_size 128 --overlap_keyframes 8) over a
     1000-frame video on the w16_320 layer: the cache restarts every 120 frames and re-streams
     the 8 overlap frames. One untimed pass, one timed pass."""
-    import paged_kv_cache_gca_b200 as gca
     from paged_kv_cache_gca_b200 import windowed
 
     w = gi.workload(WORKLOAD).replace(max_frames=window)
@@ -442,7 +649,6 @@ def run_batched_append(ring, device, stream, warm=16, timed=32):
     host enqueues the timed launches, so the events time the launches back to back."""
     import ctypes
 
-    import paged_kv_cache_gca_b200 as gca
 
     w = gi.workload("stack24x4")
     n = w.num_layers * w.num_streams
@@ -619,13 +825,17 @@ def blas_threads() -> int:
     return torch.get_num_threads()
 
 
-def oracle_frames_per_s(w: gi.Workload, sample_frames):
+def oracle_frames_per_s(w: gi.Workload, sample_frames, rows=None):
     """Oracle frames/s on this host, extrapolated from a bounded sample: bookkeeping is timed
-    over the whole stream; attention on the sampled frames (all rows, all heads) gives a cost
-    per query-key pair that is applied to every frame's T x Nk(t)."""
-    t_book, t_att = oracle_sample(w, sample_frames)
+    over the whole stream; attention on the sampled frames (all rows, or `rows` random rows;
+    all heads) gives a cost per query-key pair that is applied to every frame's T x Nk(t)."""
+    sel = None
+    if rows is not None:
+        sel = np.sort(np.random.default_rng(5).choice(w.tokens_per_frame, rows, replace=False))
+    t_book, t_att = oracle_sample(w, sample_frames, sel)
     T = w.tokens_per_frame
-    sampled_pairs = sum(T * visible_keys(w, t) for t in sample_frames)
+    n_rows = T if rows is None else rows
+    sampled_pairs = sum(n_rows * visible_keys(w, t) for t in sample_frames)
     all_pairs = sum(T * visible_keys(w, t) for t in range(w.frames))
     est = t_book + t_att * all_pairs / sampled_pairs
     return w.frames / est, {
@@ -676,6 +886,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--main-only", action="store_true",
+                    help="only the 320-frame stream and its sub-measurements (no config lines)")
     ap.add_argument("--clocks-csv", default=None,
                     help="also write the raw nvidia-smi clock samples of the timed region here")
     args = ap.parse_args()
@@ -704,8 +916,10 @@ def main():
     w, r = run_ours(args, rank, world, device)
     pk, pk_kind = peaks()
     value = aggregate_frames_per_s(world, args.steps, r["frames"], r["elapsed_ms"])
-    att_tflops = r["flops_per_step"] / (r["attend_ms_per_step"] / 1e3) / 1e12
-    peak_t = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    burst = pk["bf16_tflops"]
+    attn_tflops = r["flops_per_step"] / (r["attn_ms_per_step"] / 1e3) / 1e12
+    call_tflops = r["flops_per_step"] / ((r["attn_ms_per_step"] + r["combine_ms_per_step"])
+                                         / 1e3) / 1e12
     att_traffic = traffic_from_profile("attn")
     T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
     append_bytes = 6.0 * T * H * D * 2
@@ -713,6 +927,9 @@ def main():
     evictions = max(0, w.frames - w.anchor_frames - w.window_frames)
     app_bytes_step = append_bytes * w.frames + evict_bytes * evictions
     app_gbs = app_bytes_step / (r["append_ms_per_step"] / 1e3) / 1e9
+    plain_us = 1e3 * r["elapsed_ms"] / (args.steps * w.frames)
+    reatt_us = 1e3 * r["reattend_ms_per_step"] / w.frames
+    # combine: algorithmic bytes = the partial records read + the output rows written
     line = {
         "metric": METRIC,
         "value": value,
@@ -733,16 +950,23 @@ def main():
             "l2": "inputs larger than L2: 64-frame q/k/v ring (395 MB) on the device",
             "parallelism": "replicas" if world > 1 else "single GPU",
         },
-        "attention_tflops": att_tflops,
-        "attention_frac_of_bf16_peak": att_tflops / peak_t,
+        "attention_tflops": attn_tflops,
+        "attention_frac_of_bf16_peak": attn_tflops / burst,
         "roofline": {
-            "kernel": "gca_attend (tcgen05 paged attention + split-KV combine)",
-            "bound": "tensor", "achieved": att_tflops, "peak": peak_t, "unit": "TFLOP/s",
-            "frac": att_tflops / peak_t,
-            "peak_kind": f"bf16 sustained, {pk_kind}",
-            "frac_of_burst_peak": att_tflops / pk["bf16_tflops"],
+            "kernel": "attn_kernel (tcgen05 paged attention, one launch per frame)",
+            "bound": "tensor", "achieved": attn_tflops, "peak": burst, "unit": "TFLOP/s",
+            "frac": attn_tflops / burst,
+            "peak_kind": f"bf16 burst, {pk_kind} (each launch is timed alone, ~0.1 ms)",
+            "frac_of_sustained_peak": attn_tflops / pk.get("bf16_tflops_sustained", burst),
             "traffic": att_traffic,
             "flops_per_step": r["flops_per_step"],
+            "us_per_launch": 1e3 * r["attn_ms_per_step"] / w.frames,
+        },
+        "combine": {
+            "kernel": "combine_kernel (split-KV merge)",
+            "us_per_launch": 1e3 * r["combine_ms_per_step"] / w.frames,
+            "attend_call_tflops": call_tflops,
+            "attend_call_frac_of_burst": call_tflops / burst,
         },
         "append_roofline": {
             "kernel": "gca_append_frame (RoPE + paged scatter + eviction)",
@@ -750,12 +974,15 @@ def main():
             "frac": app_gbs / pk["hbm_gbs"], "peak_kind": pk_kind,
             "bytes_per_step": app_bytes_step,
             "us_per_append": 1e3 * r["append_ms_per_step"] / w.frames,
+            "exposed_us_per_frame": 2 * plain_us - reatt_us,
+            "exposed_how": ("(2 x plain frame time - frame time of a pass that attends every "
+                            "frame twice): the time the append adds to a frame"),
         },
         "e2e": r["e2e"],
         "gpu_launches": r["launches_per_step"] * args.steps,
         "clocks": r["clocks"],
     }
-    b = r["batched_append"]
+    b = r.get("batched")
     if b is not None:
         line["append_batch_roofline"] = {
             "kernel": "gca_append_frames (one launch over 96 caches)", "bound": "hbm",
@@ -763,20 +990,18 @@ def main():
             "frac": b["gbs"] / pk["hbm_gbs"], "peak_kind": pk_kind,
             **{k: v for k, v in b.items() if k != "gbs"},
         }
-    if r["prefill"] is not None:
+    if r.get("prefill") is not None:
         pf = r["prefill"]
         line["prefill_roofline"] = {
             "kernel": "gca_attend_prefill (tcgen05 attention, 8032 queries, + combine)",
-            "bound": "tensor", "achieved": pf["tflops"], "peak": peak_t, "unit": "TFLOP/s",
-            "frac": pf["tflops"] / peak_t, "peak_kind": f"bf16 sustained, {pk_kind}",
+            "bound": "tensor", "achieved": pf["tflops"], "peak": burst, "unit": "TFLOP/s",
+            "frac": pf["tflops"] / burst, "peak_kind": f"bf16 burst, {pk_kind}",
             **{k: v for k, v in pf.items() if k != "tflops"},
         }
-    if r["keyframes"] is not None:
-        line["keyframe_stream"] = r["keyframes"]
-    if r["camera"] is not None:
-        line["camera_head"] = r["camera"]
-    if r["windowed"] is not None:
-        line["windowed_mode"] = r["windowed"]
+    for key, name in (("keyframes", "keyframe_stream"), ("camera", "camera_head"),
+                      ("windowed", "windowed_mode"), ("configs", "configs")):
+        if r.get(key) is not None:
+            line[name] = r[key]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, d = oracle_frames_per_s(w, [w.frames // 2, w.frames - 1])
         line["cpu_baseline"] = {

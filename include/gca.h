@@ -262,6 +262,13 @@ gca_status gca_check(gca_cache* cache);
  * measurement: they show which paths of the online softmax a stream exercised). */
 gca_status gca_read_attend_counters(gca_cache* cache, gca_attend_counters* counters);
 
+/* Measurement hook: while cuda_event (a cudaEvent_t created by the caller) is set, every
+ * gca_attend / gca_attend_prefill of this cache records it on the call's stream right after the
+ * attention kernel's launch and before the combine's, so that events around the call split its
+ * time between the two kernels. NULL clears it. An event between the launches stops the combine
+ * from starting early (programmatic launch), so use it in a separate, instrumented pass. */
+gca_status gca_set_split_event(gca_cache* cache, void* cuda_event);
+
 /* Bound of every pipeline wait inside this cache's attention kernels, in nanoseconds (0 restores
  * the default, 2 s). A wait that runs out -- which only a stalled pipeline can cause -- sets
  * GCA_DEVERR_WAIT_TIMEOUT in the sticky device error word; the kernel's CTAs then stop issuing

@@ -21,7 +21,7 @@ __all__ = [
     "gca_append_frame_ex", "gca_rollback_last_frame", "gca_attend_prefill",
     "GCA_APPEND_TRANSIENT", "GcaCache", "config_for", "EXPORTED_SYMBOLS",
     "gca_set_wait_limit", "gca_test_withhold_copies", "gca_read_attend_counters",
-    "GcaAttendCounters",
+    "GcaAttendCounters", "gca_set_split_event",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -92,6 +92,7 @@ EXPORTED_SYMBOLS = (
     "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc", "gca_append_frames",
     "gca_append_frame_ex", "gca_rollback_last_frame", "gca_attend_prefill",
     "gca_set_wait_limit", "gca_test_withhold_copies", "gca_read_attend_counters",
+    "gca_set_split_event",
 )
 
 _lib = None
@@ -129,6 +130,7 @@ def lib():
         "gca_set_wait_limit": (I32, [VP, ctypes.c_uint64]),
         "gca_test_withhold_copies": (I32, [VP]),
         "gca_read_attend_counters": (I32, [VP, P(GcaAttendCounters)]),
+        "gca_set_split_event": (I32, [VP, VP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -215,6 +217,11 @@ def gca_read_attend_counters(handle) -> GcaAttendCounters:
     out = GcaAttendCounters()
     _ok(lib().gca_read_attend_counters(handle, ctypes.byref(out)), "gca_read_attend_counters")
     return out
+
+
+def gca_set_split_event(handle, cuda_event) -> None:
+    """cuda_event: a cudaEvent_t handle (int, e.g. torch.cuda.Event().cuda_event) or None."""
+    _ok(lib().gca_set_split_event(handle, cuda_event), "gca_set_split_event")
 
 
 def gca_reset(handle, stream) -> None:

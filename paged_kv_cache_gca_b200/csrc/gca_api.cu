@@ -540,6 +540,7 @@ gca_status enqueue_attention(gca_cache* c, int64_t t, int64_t q_rows, const void
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (launch_attn(c->tm_k, c->tm_v, p, s) != cudaSuccess) return GCA_ERR_CUDA;
   c->withhold_next = 0;
+  if (c->split_event && cudaEventRecord(c->split_event, s) != cudaSuccess) return GCA_ERR_CUDA;
   if (split && launch_combine(p, s) != cudaSuccess) return GCA_ERR_CUDA;
 
   gca_attend_info& inf = c->last;
@@ -659,6 +660,12 @@ gca_status gca_read_attend_counters(gca_cache* c, gca_attend_counters* out) {
   out->exact_max_rows = v[0];
   out->rescaled_rows = v[1];
   out->wide_merge_rows = v[2];
+  return GCA_OK;
+}
+
+gca_status gca_set_split_event(gca_cache* c, void* cuda_event) {
+  if (!c) return GCA_ERR_INVALID_ARG;
+  c->split_event = static_cast<cudaEvent_t>(cuda_event);
   return GCA_OK;
 }
 

@@ -248,6 +248,7 @@ struct gca_cache {
   uint32_t dev_err;
   uint64_t wait_ns;        // attention wait bound (gca_set_wait_limit)
   int32_t withhold_next;   // test hook armed for the next attention launch
+  cudaEvent_t split_event; // measurement hook: recorded between attention and combine launches
   CUtensorMap tm_k;
   CUtensorMap tm_v;
   gca_attend_info last;
