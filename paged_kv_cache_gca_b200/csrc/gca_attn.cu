@@ -22,10 +22,11 @@
 // CTA roles (352 threads):
 //   warps 0-3, 4-7  softmax warpgroup of query tile 0 / 1: thread r owns query row r (TMEM lane
 //              r). Loads its Q tile into swizzled shared memory; per key tile reads S from TMEM,
-//              masks unused page slots, takes the row max, computes P = 2^(s*log2e/sqrt(D) - m)
-//              (FFMA + MUFU ex2), writes P as bf16 over the first half of the same TMEM buffer
-//              and accumulates the row sum. O in TMEM is rescaled only when the row max grows by
-//              more than 2^8 (lazy rescale).
+//              masks unused page slots, takes the row max, then -- taking turns with the other
+//              warpgroup, because the exponentials are the bottleneck (MUFU) -- computes
+//              P = 2^(s*log2e/sqrt(D) - m) (FFMA + MUFU ex2), writes P as bf16 over the first
+//              half of the same TMEM buffer and accumulates the row sum. O in TMEM is rescaled
+//              only when the row max grows by more than 2^8 (lazy rescale).
 //   warp 8     TMA producer: resolves the tile's 6 page ids and issues 12 page copies (K, V)
 //              per tile into 4-stage K and V rings.
 //   warps 9,10 MMA issuers, one per query tile: S(j) = Q K_j^T (A, B from shared memory) into
@@ -83,6 +84,7 @@ struct __align__(8) Shared {
   uint64_t p_full[kQPerCta][2];   // P(j) of query tile q written over buffer j % 2
   uint64_t pv_done[kQPerCta][2];  // O += P(j) V_j of query tile q has completed
   uint64_t mma_drain[kQPerCta];   // every MMA of query tile q has completed (teardown)
+  uint64_t turn[kQPerCta];        // exponential turns of the two softmax warpgroups
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -475,9 +477,15 @@ __device__ __forceinline__ void softmax_group(const AttnParams& p, Shared& sh, u
   const int r = (warp & 3) * 32 + lane;
   const uint32_t t_row = tmem + kTmemPerQ * qq + ((uint32_t)((warp & 3) * 32) << 16);
   uint8_t* q_tile = q_smem + qq * kQTileBytes;
-  uint32_t it = 0;
+  uint32_t it = 0, turns = 0;
   uint32_t n_exact = 0, n_rescale = 0;  // branch counts of this row (past each first tile)
   bool ok = true;
+  // The two warpgroups take turns for the exponentials (MUFU-bound): while one computes them,
+  // the other waits for its next S, loads it and reduces the row max, so the two stay half a
+  // tile apart instead of stalling on their loads at the same time. Query tile 0 goes first.
+  uint64_t* const my_turn = &sh.turn[qq];
+  uint64_t* const their_turn = &sh.turn[qq ^ 1];
+  if (qq == 1) mbar_arrive(their_turn);
   for (int64_t s = s_begin; s < s_end && ok;) {
     const int u2 = (int)(s / p.n_tiles);
     const int64_t seg_end = min(s_end, (int64_t)(u2 + 1) * p.n_tiles);
@@ -588,8 +596,12 @@ __device__ __forceinline__ void softmax_group(const AttnParams& p, Shared& sh, u
           tmem_st16(t_row + kColO + 16 * c, o);
         }
       }
-      // P = 2^(s*c - m): scale-subtract, exponentials, bf16 packing, row sum; P goes to the
-      // first 48 columns of the buffer S came from (S is dead once loaded).
+      // P = 2^(s*c - m), in this warpgroup's turn: scale-subtract, exponentials, bf16
+      // packing, row sum; P goes to the first 48 columns of the buffer S came from (S is dead
+      // once loaded). The turn passes to the other warpgroup one 32-column chunk before the
+      // end, so that its first exponentials queue behind this group's last ones.
+      if (!warp_wait<true>(my_turn, turns & 1u, &sh, p)) { ok = false; break; }
+      ++turns;
       const float neg_m = -m_new;
 #pragma unroll
       for (int e = 0; e < kTileK; ++e) sv[e] = fmaf(sv[e], p.scale_log2, neg_m);
@@ -609,6 +621,7 @@ __device__ __forceinline__ void softmax_group(const AttnParams& p, Shared& sh, u
           rs[2 * (c & 3) + 1] += e1;
         }
         tmem_st16(t_buf + 16 * chunk, reinterpret_cast<const float*>(pk));
+        if (chunk == kTileK / 32 - 2) mbar_arrive(their_turn);
       }
       const float row_sum =
           ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
@@ -692,6 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int q = 0; q < kQPerCta; ++q) {
       mbar_init(&sh.q_full[q], kTileQ);
       mbar_init(&sh.mma_drain[q], 1);
+      mbar_init(&sh.turn[q], kTileQ);
       for (int b = 0; b < 2; ++b) {
         mbar_init(&sh.s_full[q][b], 1);
         mbar_init(&sh.p_full[q][b], kTileQ);

