@@ -326,9 +326,30 @@ __device__ __forceinline__ void resolve_page(const AttnParams& p, int lp, int fa
   }
 }
 
+// Page ids of kBatchTiles consecutive steps, fetched in one round of loads: lane l <
+// kBatchTiles * kPagesPerTile holds page l % kPagesPerTile of step s0 + l / kPagesPerTile (the
+// logical pages of a key tile do not depend on the work unit, only on the tile index).
+constexpr int kBatchTiles = 5;
+static_assert(kBatchTiles * kPagesPerTile <= 32, "one page per lane");
+struct PageBatch {
+  int page, len;
+};
+
+__device__ __forceinline__ PageBatch fetch_pages(const AttnParams& p, int64_t s0, int64_t s_end,
+                                                 int fallback, int lane) {
+  PageBatch b{fallback, 0};
+  const int64_t s = s0 + lane / kPagesPerTile;
+  if (lane < kBatchTiles * kPagesPerTile && s < s_end) {
+    const int j = (int)(s % p.n_tiles);
+    resolve_page(p, j * kPagesPerTile + lane % kPagesPerTile, fallback, &b.page, &b.len);
+  }
+  return b;
+}
+
 // ------------------------------------------------------------------------- roles
 
-// Warp 8: resolves each tile's pages and issues their K and V copies.
+// Warp 8: resolves each tile's pages and issues their K and V copies. The page ids are fetched
+// kBatchTiles steps ahead of their use, so the page-table loads never stall the copies.
 __device__ __forceinline__ void tma_producer(const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                              const AttnParams& p, Shared& sh, uint8_t* k_smem,
                                              uint8_t* v_smem, int64_t s_begin, int64_t s_end) {
@@ -341,6 +362,8 @@ __device__ __forceinline__ void tma_producer(const CUtensorMap* tm_k, const CUte
   // test hook: CTA 0 never issues the copies of its first tile, so the MMA issuer's wait for
   // them runs out (nothing is in flight for that tile at any time)
   const bool withhold_first = p.withhold != 0 && blockIdx.x == 0;
+  PageBatch cur = fetch_pages(p, s_begin, s_end, fallback, lane);
+  PageBatch nxt = fetch_pages(p, s_begin + kBatchTiles, s_end, fallback, lane);
   for (int64_t s = s_begin; s < s_end && ok;) {
     const int u2 = (int)(s / p.n_tiles);
     const int64_t seg_end = min(s_end, (int64_t)(u2 + 1) * p.n_tiles);
@@ -349,9 +372,14 @@ __device__ __forceinline__ void tma_producer(const CUtensorMap* tm_k, const CUte
     for (int j = (int)(s - (int64_t)u2 * p.n_tiles); j < j_end; ++j, ++it) {
       const int st = it % kStages;
       const uint32_t use = it / kStages;
-      int page = 0, len = 0;
-      if (lane < kPagesPerTile) resolve_page(p, j * kPagesPerTile + lane, fallback, &page, &len);
-      if (page < 0 || page >= p.num_pages) {
+      const int kb = (int)(it % kBatchTiles);
+      if (kb == 0 && it > 0) {
+        cur = nxt;
+        nxt = fetch_pages(p, s_begin + it + kBatchTiles, s_end, fallback, lane);
+      }
+      int page = __shfl_sync(0xffffffffu, cur.page, kb * kPagesPerTile + lane % kPagesPerTile);
+      int len = __shfl_sync(0xffffffffu, cur.len, kb * kPagesPerTile + lane % kPagesPerTile);
+      if (lane < kPagesPerTile && (page < 0 || page >= p.num_pages)) {
         atomicOr(p.err, GCA_DEVERR_PAGE_RANGE);
         page = 0;
         len = 0;

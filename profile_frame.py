@@ -1,19 +1,20 @@
-"""Positions one cache at frame t of a workload and runs gca_attend there once.
+"""Profiling helper of the benchmark: positions one cache at frame t of a workload and runs
+gca_attend there.
 
 For profilers: the appends of frames 0..t run first (cheap kernels), then exactly `--repeat`
 attention calls at frame t, so a capture can select them with few launches before them.
 
-    python -m paged_kv_cache_gca_b200.profile_frame --workload w16_320 --frame 319 --repeat 1
+    python profile_frame.py --workload w16_320 --frame 319 --repeat 1
 
 With --batch N it instead creates N caches of the workload and runs --frame + 1 batched appends
 (gca_append_frames over all N caches; frame of cache c at step t: ring slot (N t + c) mod R):
 
-    python -m paged_kv_cache_gca_b200.profile_frame --workload stack24x4 --batch 16 --frame 15
+    python profile_frame.py --workload stack24x4 --batch 16 --frame 15
 
 With --prefill it appends the workload's anchor (scale) frames and runs --repeat joint
 attentions over them (gca_attend_prefill):
 
-    python -m paged_kv_cache_gca_b200.profile_frame --workload scale8 --prefill --repeat 1
+    python profile_frame.py --workload scale8 --prefill --repeat 1
 """
 import argparse
 import os
@@ -21,7 +22,7 @@ import sys
 
 import torch
 
-ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
