@@ -296,9 +296,6 @@ def run_ours(args, rank, world, device):
     e2e = run_e2e(args, w, cache, ring_host, device, stream, world)
     extra = {}
     if world == 1:
-        plain_us = 1e3 * elapsed_ms / (args.steps * nframes)
-        attention_us = 1e3 * re_ms / (args.steps * nframes) - plain_us  # attention's own time
-        extra["fused"] = run_fused_stream(ring, device, stream, args.steps, attention_us)
         extra["batched"] = run_batched_append(ring, device, stream)
         extra["prefill"] = run_prefill(ring, device, stream)
         extra["keyframes"] = run_keyframe_stream(ring, device, stream)
@@ -322,57 +319,6 @@ def run_ours(args, rank, world, device):
     }
     cache.close()
     return w, res
-
-
-def run_fused_stream(ring, device, stream, steps, reattend_us):
-    """The 320-frame stream through gca_append_attend (append and attention of a frame in one
-    launch): frames/s, and the attention kernel's time per launch with events around it."""
-    w = gi.workload(WORKLOAD)
-    T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
-    with torch.cuda.stream(stream):
-        cache = gca.GcaCache(gca.config_for(w), initial_free=gi.initial_free_list(w),
-                             stream=stream)
-    out = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
-    flops = []
-
-    def one_step(ev=None):
-        cache.reset(stream=stream)
-        for t in range(w.frames):
-            q, k, v = ring[t % w.ring]
-            if ev is not None:
-                ev[t][0].record(stream)
-                ev[t][1].record(stream)
-                gca.gca_set_split_event(cache.handle, ev[t][2].cuda_event)
-            cache.append_attend(t, q, k, v, out, stream=stream)
-            if ev is not None:
-                ev[t][3].record(stream)
-            if len(flops) < w.frames:
-                flops.append(attn_flops(w, cache.attend_info().visible_keys))
-        if ev is not None:
-            gca.gca_set_split_event(cache.handle, None)
-
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            one_step()
-    ms = timed(stream, lambda: [one_step() for _ in range(steps)]) / steps
-    ev = new_events(w.frames)
-    with torch.cuda.stream(stream):
-        one_step(ev)
-    torch.cuda.synchronize()
-    _, k, c = split_times(ev, range(w.frames))
-    assert cache.check() == 0, "device error in the fused stream"
-    cache.close()
-    frame_us = 1e3 * ms / w.frames
-    return {"workload": f"{w.name} through gca_append_attend (one launch per frame for append "
-                        "and attention, + combine)",
-            "frames_per_s": w.frames / (ms / 1e3), "ms_per_step": ms,
-            "attention_tflops_stream": sum(flops) / (ms / 1e3) / 1e12,
-            "fused_kernel_us_per_launch": 1e3 * k / w.frames,
-            "fused_kernel_tflops": sum(flops) / (k / 1e3) / 1e12,
-            "combine_us_per_launch": 1e3 * c / w.frames,
-            "append_exposed_us_per_frame": frame_us - reattend_us,
-            "exposed_how": ("fused frame time - the attention's own time per frame (a plain "
-                            "pass of the separate calls that attends every frame twice)")}
 
 
 def run_stream_config(w, device, stream, warm=1, timed_passes=1, span=None, events=True):
@@ -1052,8 +998,7 @@ def main():
             "frac": pf["tflops"] / burst, "peak_kind": f"bf16 burst, {pk_kind}",
             **{k: v for k, v in pf.items() if k != "tflops"},
         }
-    for key, name in (("fused", "fused_stream"), ("keyframes", "keyframe_stream"),
-                      ("camera", "camera_head"),
+    for key, name in (("keyframes", "keyframe_stream"), ("camera", "camera_head"),
                       ("windowed", "windowed_mode"), ("configs", "configs")):
         if r.get(key) is not None:
             line[name] = r[key]

@@ -212,21 +212,6 @@ gca_status gca_append_frames(gca_cache* const* caches, int32_t n, const int64_t*
 gca_status gca_attend(gca_cache* cache, int64_t frame_idx, const void* q_rot, void* out,
                       void* stream);
 
-/* gca_append_frame followed by gca_attend of the same frame, in ONE kernel launch (+ one
- * combine launch when the key range is split): while most warps of the attention kernel attend
- * over the keys the append does not touch, one warp per CTA performs the append (RoPE, paged
- * scatter of k and v, eviction) and the frame's queries are rotated as they are loaded. Key
- * tiles that hold the frame's own pages or the trajectory pages receiving kept tokens are
- * processed last, once the append is complete. Same pool contents, page tables and free list as
- * the two calls (bit-identical); the attention equals gca_attend's up to the rounding of a
- * different order of key tiles. q, k, v: device bf16 [T][H][D] (raw, unrotated); out: device
- * bf16 [T][H][D], not overlapping q, k or v (GCA_ERR_INVALID_ARG). No q_rot is written.
- * frame_idx and errors as gca_append_frame (checked on the host, nothing enqueued on error);
- * GCA_ERR_UNSUPPORTED as gca_attend. Once the cache's sticky device error is set the launch
- * does nothing, the append included, until gca_reset. */
-gca_status gca_append_attend(gca_cache* cache, int64_t frame_idx, const void* q, const void* k,
-                             const void* v, void* out, void* stream);
-
 /* Joint attention of the first n frames (the scale frames), bidirectional: after exactly n
  * appends (n <= anchor_frames, so all n frames are anchors), the n*T queries of frames 0..n-1
  * attend over every token of those frames, with no mask across frames (pages: the scale frames

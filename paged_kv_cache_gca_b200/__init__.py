@@ -21,7 +21,7 @@ __all__ = [
     "gca_append_frame_ex", "gca_rollback_last_frame", "gca_attend_prefill",
     "GCA_APPEND_TRANSIENT", "GcaCache", "config_for", "EXPORTED_SYMBOLS",
     "gca_set_wait_limit", "gca_test_withhold_copies", "gca_read_attend_counters",
-    "GcaAttendCounters", "gca_set_split_event", "gca_append_attend",
+    "GcaAttendCounters", "gca_set_split_event",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -92,7 +92,7 @@ EXPORTED_SYMBOLS = (
     "gca_last_attend_info", "gca_status_string", "gca_attend_noalloc", "gca_append_frames",
     "gca_append_frame_ex", "gca_rollback_last_frame", "gca_attend_prefill",
     "gca_set_wait_limit", "gca_test_withhold_copies", "gca_read_attend_counters",
-    "gca_set_split_event", "gca_append_attend",
+    "gca_set_split_event",
 )
 
 _lib = None
@@ -131,7 +131,6 @@ def lib():
         "gca_test_withhold_copies": (I32, [VP]),
         "gca_read_attend_counters": (I32, [VP, P(GcaAttendCounters)]),
         "gca_set_split_event": (I32, [VP, VP]),
-        "gca_append_attend": (I32, [VP, I64, VP, VP, VP, VP, VP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -183,12 +182,6 @@ def gca_rollback_last_frame(handle, frame_idx, stream=None) -> None:
 
 def gca_attend_prefill(handle, n, q_rot_ptr, out_ptr, stream) -> None:
     _ok(lib().gca_attend_prefill(handle, n, q_rot_ptr, out_ptr, stream), "gca_attend_prefill")
-
-
-def gca_append_attend(handle, frame_idx, q_ptr, k_ptr, v_ptr, out_ptr, stream) -> None:
-    """Append and attention of one frame in one launch (raw q, k, v)."""
-    _ok(lib().gca_append_attend(handle, frame_idx, q_ptr, k_ptr, v_ptr, out_ptr, stream),
-        "gca_append_attend")
 
 
 def gca_attend(handle, frame_idx, q_rot_ptr, out_ptr, stream) -> None:
@@ -317,11 +310,6 @@ class GcaCache:
                                 GCA_APPEND_TRANSIENT if transient else 0, q.data_ptr(),
                                 k.data_ptr(), v.data_ptr(), q_rot.data_ptr(),
                                 _stream_handle(stream))
-
-    def append_attend(self, t, q, k, v, out, stream=None):
-        """Appends frame t and attends its queries in one launch (raw q, k, v)."""
-        gca_append_attend(self.handle, t, q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                          out.data_ptr(), _stream_handle(stream))
 
     def rollback(self, t):
         gca_rollback_last_frame(self.handle, t)

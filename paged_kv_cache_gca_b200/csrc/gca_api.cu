@@ -149,7 +149,6 @@ bool compute_layout(const gca_config& c, Layout* L) {
   L->err = take(4);
   L->kmax = take(4 * (size_t)c.num_heads);
   L->counters = take(8 * 4);
-  L->step_counters = take(8 * 4);
   L->part_o = take(4 * (size_t)L->part_slots * kTileQ * kHeadDim);
   L->part_ml = take(8 * (size_t)L->part_slots * kTileQ);
   L->total = align_up(off, kAlign);
@@ -207,7 +206,6 @@ bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams
   g = std::min<int64_t>(g, p->total);
   p->grid = (int32_t)g;
   p->scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)cf.head_dim));
-  p->dep_a = p->dep_b = p->dep_c = p->n_tiles;  // nothing waits for an append
   p->wait_ns = c->wait_ns > 0 ? c->wait_ns : kDefaultWaitNs;
   p->withhold = c->withhold_next;
   bool sp = false;
@@ -329,8 +327,7 @@ gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t w
             cudaMemsetAsync(c->ws + L.seen, 0, 4 * (size_t)cfg->num_pages, s) == cudaSuccess &&
             cudaMemsetAsync(c->ws + L.err, 0, 4, s) == cudaSuccess &&
             cudaMemsetAsync(c->ws + L.kmax, 0, 4 * (size_t)cfg->num_heads, s) == cudaSuccess &&
-            cudaMemsetAsync(c->ws + L.counters, 0, 8 * 4, s) == cudaSuccess &&
-            cudaMemsetAsync(c->ws + L.step_counters, 0, 8 * 4, s) == cudaSuccess;
+            cudaMemsetAsync(c->ws + L.counters, 0, 8 * 4, s) == cudaSuccess;
   if (ok) {
     InitParams ip;
     std::memset(&ip, 0, sizeof(ip));
@@ -370,15 +367,14 @@ gca_status gca_cache_create(const gca_config* cfg, void* dev_workspace, size_t w
 namespace {
 
 // Checks one append and fills its launch parameters from the host mirror; changes nothing.
-// q_rot_out may be null only for the fused call (its queries are rotated as they are loaded).
 gca_status prepare_append(gca_cache* c, int64_t t, int64_t rope_frame, uint32_t flags,
                           const void* q, const void* k, const void* v, void* q_rot_out,
-                          AppendParams* out, bool fused = false) {
-  if (!c || !q || !k || !v || (!q_rot_out && !fused)) return GCA_ERR_INVALID_ARG;
+                          AppendParams* out) {
+  if (!c || !q || !k || !v || !q_rot_out) return GCA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_rot_out)) {
     return GCA_ERR_INVALID_ARG;
   }
-  if (q_rot_out) {
+  {
     // Each thread reads its own chunk of q, k, v and writes the same chunk of q_rot, so q_rot
     // may be q itself; any other overlap with q, k or v would let a thread overwrite a chunk
     // another thread has yet to read.
@@ -584,76 +580,6 @@ gca_status gca_attend_prefill(gca_cache* c, int32_t n, const void* q_rot, void* 
   return enqueue_attention(c, n - 1, (int64_t)n * c->lay.T, q_rot, out, stream);
 }
 
-gca_status gca_append_attend(gca_cache* c, int64_t t, const void* q, const void* k,
-                             const void* v, void* out, void* stream) {
-  NvtxRange range_("gca_append_attend");
-  if (!c || !out || !aligned16(out)) return GCA_ERR_INVALID_ARG;
-  {
-    // the append reads k and v and the attention reads q while other CTAs write output rows
-    const size_t bytes = (size_t)c->lay.T * c->cfg.num_heads * kHeadDim * 2;
-    if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes)) {
-      return GCA_ERR_INVALID_ARG;
-    }
-  }
-  AppendParams ap;
-  gca_status st = prepare_append(c, t, t, 0u, q, k, v, nullptr, &ap, true);
-  if (st != GCA_OK) return st;
-  // the attention plan sees the state after this frame's append
-  const gca_cache saved = *c;
-  commit_append(c, ap, false);
-  const Layout& L = c->lay;
-  AttnParams p;
-  bool split = false;
-  int64_t nk = 0;
-  if (!plan_attention(c, t, L.part_slots, &p, &split, &nk)) {
-    *c = saved;
-    return GCA_ERR_UNSUPPORTED;
-  }
-  p.q = static_cast<const uint4*>(q);
-  p.out = static_cast<uint4*>(out);
-  p.part_o = at<float>(c, L.part_o);
-  p.part_ml = at<float2>(c, L.part_ml);
-  p.fused = 1;
-  p.ap = ap;
-  p.append_items = (int64_t)ap.ppf * kPageSize * ap.H * 8 + ap.n_aux_items;
-  unsigned long long* sc = at<unsigned long long>(c, L.step_counters);
-  const int slot = (int)(c->fused_launches & 1);
-  p.claim = sc + 2 * slot;
-  p.done = sc + 2 * slot + 1;
-  p.next_counters = sc + 2 * (slot ^ 1);
-  // Key tiles that read what this append writes: the frame's own pages (the last ppf logical
-  // pages before the trajectory) and, when a frame is evicted, the trajectory from the page
-  // that receives its kept tokens on.
-  const int32_t frame_end = p.na_pages + p.nw_pages;
-  p.dep_a = (frame_end - L.ppf) / kPagesPerTile;
-  p.dep_b = (frame_end + kPagesPerTile - 1) / kPagesPerTile;
-  p.dep_c = p.n_tiles;
-  if (ap.K > 0) {
-    const int32_t first_traj = frame_end + (int32_t)(ap.traj_len / kPageSize);
-    p.dep_c = std::min<int32_t>(p.n_tiles, first_traj / kPagesPerTile);
-  }
-  if (p.dep_c < p.dep_b) p.dep_b = p.dep_c;  // [dep_a, dep_b) and [dep_c, ...) meet
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (launch_attn(c->tm_k, c->tm_v, p, s) != cudaSuccess) {
-    *c = saved;
-    return GCA_ERR_CUDA;
-  }
-  c->withhold_next = 0;
-  c->fused_launches += 1;
-  if (c->split_event && cudaEventRecord(c->split_event, s) != cudaSuccess) return GCA_ERR_CUDA;
-  if (split && launch_combine(p, s) != cudaSuccess) return GCA_ERR_CUDA;
-  gca_attend_info& inf = c->last;
-  inf.frame_idx = t;
-  inf.visible_keys = nk;
-  inf.logical_pages = p.n_lp;
-  inf.kv_tiles = p.n_tiles;
-  inf.query_tiles = p.n_qt;
-  inf.grid = p.grid;
-  inf.split = split ? 1 : 0;
-  inf.launches = split ? 2 : 1;
-  return GCA_OK;
-}
-
 gca_status gca_reset(gca_cache* c, void* stream) {
   NvtxRange range_("gca_reset");
   if (!c) return GCA_ERR_INVALID_ARG;
@@ -665,8 +591,6 @@ gca_status gca_reset(gca_cache* c, void* stream) {
       cudaMemsetAsync(c->ws + L.kmax, 0, 4 * (size_t)c->cfg.num_heads,
                       static_cast<cudaStream_t>(stream)) != cudaSuccess ||
       cudaMemsetAsync(c->ws + L.counters, 0, 8 * 4, static_cast<cudaStream_t>(stream)) !=
-          cudaSuccess ||
-      cudaMemsetAsync(c->ws + L.step_counters, 0, 8 * 4, static_cast<cudaStream_t>(stream)) !=
           cudaSuccess) {
     return GCA_ERR_CUDA;
   }
@@ -677,7 +601,6 @@ gca_status gca_reset(gca_cache* c, void* stream) {
   c->traj_pages = 0;
   c->transient = false;
   c->dev_err = 0;
-  c->fused_launches = 0;
   std::memset(&c->last, 0, sizeof(c->last));
   return GCA_OK;
 }

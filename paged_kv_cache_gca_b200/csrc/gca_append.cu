@@ -130,9 +130,26 @@ __device__ __forceinline__ void append_block(const AppendParams& p, const int bx
 // slower).
 #define GCA_APPEND_BOUNDS __launch_bounds__(512, 4)
 
-__global__ void GCA_APPEND_BOUNDS append_kernel(const AppendParams p) {
+// One frame's append: warp w of the grid takes token items [128 w, 128 w + 128), four per lane
+// with their loads in flight together (a single 12 MB frame is one short wave, so memory-level
+// parallelism per thread, not occupancy, bounds it); the warps after the token items take the
+// eviction items, one per lane.
+constexpr int kAppendWarpsPerBlock = 8;
+constexpr int kItemsPerWarp = 128;
+
+__global__ void __launch_bounds__(32 * kAppendWarpsPerBlock)
+    append_kernel(const AppendParams p) {
   pdl_wait();  // inputs, pages and the free ring may come from earlier work in the stream
-  append_block(p, (int)blockIdx.x);
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (int64_t)blockIdx.x * kAppendWarpsPerBlock + (threadIdx.x >> 5);
+  const int64_t n_tok = (int64_t)p.ppf * kPageSize * p.H * 8;
+  const int64_t tok_warps = n_tok / kItemsPerWarp;
+  if (warp < tok_warps) {
+    append_item::token_chunks4<true>(p, warp * kItemsPerWarp, lane);
+  } else {
+    const int64_t idx = (warp - tok_warps) * 32 + lane;
+    if (idx < p.n_aux_items) append_item::aux(p, idx);
+  }
   pdl_launch_dependents();
 }
 
@@ -168,8 +185,12 @@ cudaError_t launch_reset(int32_t* free_ring, const int32_t* init_free, uint32_t*
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
-  const dim3 block(8, p.H, p.tok_per_block);
-  return launch_dependent(append_kernel, dim3((unsigned)p.n_blocks), block, 0, s, p);
+  // token items: ppf * 16 slots x H heads x 8 chunks, a multiple of 128 since 16 * 8 = 128
+  const int64_t n_tok = (int64_t)p.ppf * kPageSize * p.H * 8;
+  const int64_t warps = n_tok / kItemsPerWarp + (p.n_aux_items + 31) / 32;
+  const int64_t blocks = (warps + kAppendWarpsPerBlock - 1) / kAppendWarpsPerBlock;
+  return launch_dependent(append_kernel, dim3((unsigned)blocks),
+                          dim3(32 * kAppendWarpsPerBlock), 0, s, p);
 }
 
 cudaError_t launch_append_batch(const AppendBatch& b, cudaStream_t s) {

@@ -1,5 +1,6 @@
-// Per-item code of the append step, shared by the append kernels (gca_append.cu) and the fused
-// append + attention launch (gca_attn.cu), so that both write bit-identical pages.
+// Per-item code of the append step, shared by the append kernels of gca_append.cu: the per-frame
+// kernel (four items per thread, loads hoisted) and the batched kernel (one item per thread) write
+// bit-identical pages.
 //
 // One frame's append ("How the Geometric Context Transformer Enables Streaming 3D Reconstruction
 // in LingBot-Map", FlashInferBlock: append_frame, then evict_frames) splits into items:
@@ -116,6 +117,84 @@ __device__ __forceinline__ void token_chunk(const AppendParams& p, int i, int h,
   ss += __shfl_xor_sync(group, ss, 2);
   ss += __shfl_xor_sync(group, ss, 4);
   if (c == 0 && ss > __uint_as_float(p.kmax[h])) atomicMax(&p.kmax[h], __float_as_uint(ss));
+}
+
+// Token items base + lane + 32 u, u = 0..3 (base a multiple of 8, all four below the token item
+// count): the same writes as four token_chunk<kWithQ> calls, with the loads of the four items
+// issued before any of their stores so that they are in flight together.
+template <bool kWithQ>
+__device__ __forceinline__ void token_chunks4(const AppendParams& p, int64_t base, int lane) {
+  const int H = p.H;
+  const int c = lane & 7;
+  int i[4], h[4], page[4];
+  uint4 qv[4], kv[4], vv[4];
+  float2 cs[4][4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int64_t th = (base + 32 * u + lane) >> 3;
+    h[u] = (int)(th % H);
+    i[u] = (int)(th / H);
+    page[u] = p.free_ring[wrap(p.head_pos + i[u] / kPageSize, p.num_pages)];
+    if (i[u] < p.T) {
+      const int64_t src = ((int64_t)i[u] * H + h[u]) * 8 + c;
+      if (kWithQ) qv[u] = p.q[src];
+      kv[u] = p.k[src];
+      vv[u] = p.v[src];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        cs[u][w] = rope_cs(p.rope_t, p.rope_tok, p.nt, p.nyx, p.rope_frame, i[u], 4 * c + w);
+      }
+    }
+  }
+  unsigned lane_id;
+  asm("mov.u32 %0, %%laneid;" : "=r"(lane_id));
+  const unsigned group = 0xffu << (lane_id & 24u);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    if (page[u] < 0 || page[u] >= p.num_pages) {
+      set_err(p.err, GCA_DEVERR_PAGE_RANGE);
+      continue;
+    }
+    const int slot = i[u] % kPageSize;
+    const int64_t dst = (((int64_t)page[u] * H + h[u]) * kPageSize + slot) * 8 + c;
+    if (i[u] >= p.T) {  // padding slot of the frame's last page
+      p.k_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
+      p.v_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    if (kWithQ) {
+      uint4 qr;
+      qr.x = rotate_word(qv[u].x, cs[u][0]);
+      qr.y = rotate_word(qv[u].y, cs[u][1]);
+      qr.z = rotate_word(qv[u].z, cs[u][2]);
+      qr.w = rotate_word(qv[u].w, cs[u][3]);
+      p.q_rot[((int64_t)i[u] * H + h[u]) * 8 + c] = qr;
+    }
+    uint4 kr;
+    kr.x = rotate_word(kv[u].x, cs[u][0]);
+    kr.y = rotate_word(kv[u].y, cs[u][1]);
+    kr.z = rotate_word(kv[u].z, cs[u][2]);
+    kr.w = rotate_word(kv[u].w, cs[u][3]);
+    if (h[u] == 0 && c == 0) {
+      p.slot_map[i[u]] = page[u] * kPageSize + slot;
+      if (slot == 0) p.frame_pages[p.t * p.ppf + i[u] / kPageSize] = page[u];
+    }
+    p.k_pool[dst] = kr;
+    p.v_pool[dst] = vv[u];
+    float ss = 0.f;
+    const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float a = bf_lo(kw[w]), b = bf_hi(kw[w]);
+      ss = fmaf(a, a, fmaf(b, b, ss));
+    }
+    ss += __shfl_xor_sync(group, ss, 1);
+    ss += __shfl_xor_sync(group, ss, 2);
+    ss += __shfl_xor_sync(group, ss, 4);
+    if (c == 0 && ss > __uint_as_float(p.kmax[h[u]])) {
+      atomicMax(&p.kmax[h[u]], __float_as_uint(ss));
+    }
+  }
 }
 
 // Aux item idx (0 <= idx < p.n_aux_items).

@@ -19,7 +19,7 @@
 // that spans several CTAs leaves partial (O, row max, row sum) records per query tile that a
 // combine kernel merges with log-sum-exp weights.
 //
-// CTA roles (384 threads):
+// CTA roles (352 threads):
 //   warps 0-3, 4-7  softmax warpgroup of query tile 0 / 1: thread r owns query row r (TMEM lane
 //              r). Loads its Q tile into swizzled shared memory; per key tile reads S from TMEM,
 //              masks unused page slots, takes the row max, then -- taking turns with the other
@@ -29,10 +29,6 @@
 //              only when the row max grows by more than 2^8 (lazy rescale).
 //   warp 8     TMA producer: resolves the tile's 6 page ids and issues 12 page copies (K, V)
 //              per tile into 4-stage K and V rings.
-//   warp 11   (fused launches, gca_append_attend) the frame's append: claims the append's items
-//              and writes K and V to their pages while the other warps attend over the keys
-//              that the append does not touch; key tiles holding the frame's own pages or the
-//              trajectory tail come last in every work piece, after the append is complete.
 //   warps 9,10 MMA issuers, one per query tile: S(j) = Q K_j^T (A, B from shared memory) into
 //              S/P buffer j % 2, then O += P(j-1) V_(j-1) with P read from TMEM (A operand in
 //              tensor memory) and V from shared memory (MN-major).
@@ -47,7 +43,7 @@
 // kernel returns.
 #include <cuda_bf16.h>
 
-#include "gca_append_item.cuh"
+#include "gca_internal.h"
 
 namespace gca {
 namespace {
@@ -56,12 +52,9 @@ constexpr int kStages = 4;          // K and V rings
 constexpr int kLensRing = 8;        // page-length words in flight (the producer leads the
                                     // softmax by at most kStages + 2 tiles)
 constexpr int kSoftmaxWarps = 4 * kQPerCta;
-// + TMA warp, MMA warps, append warp (active in fused launches only)
-constexpr int kThreads = 32 * (kSoftmaxWarps + 2 + kQPerCta);
+constexpr int kThreads = 32 * (kSoftmaxWarps + 1 + kQPerCta);  // + TMA warp + MMA warps
 constexpr int kWarpTma = kSoftmaxWarps;
 constexpr int kWarpMma0 = kSoftmaxWarps + 1;  // MMA warp of query tile q: kWarpMma0 + q
-constexpr int kWarpAppend = kSoftmaxWarps + 1 + kQPerCta;
-constexpr int kClaimItems = 128;  // append items a warp claims at a time (4 per lane)
 constexpr uint32_t kQTileBytes = kTileQ * kHeadDim * 2;      // 16 KB
 constexpr uint32_t kKvTileBytes = kTileK * kHeadDim * 2;     // 12 KB
 constexpr uint32_t kPageBytes = kPageSize * kHeadDim * 2;    // 2 KB
@@ -328,67 +321,8 @@ __device__ __forceinline__ void resolve_page(const AttnParams& p, int lp, int fa
     *page = p.traj_pages[tp];
     *len = (tp == p.n_traj_pages - 1) ? p.traj_tail_len : kPageSize;
   } else {
-    *page = fallback;  // masked slots: any page with finite data
+    *page = fallback;  // any visible page: finite data, fully masked
     *len = 0;
-  }
-}
-
-// ------------------------------------------------------------------------- step order
-
-// A CTA's steps [s_begin, s_end) are its work pieces ("segments": consecutive key tiles of one
-// work unit), taken in reverse order (the last unit first), and within a piece the key tiles
-// that do not depend on a fused append come first (ascending), then the dependent ones
-// (ascending). The order of a row's key tiles does not change its softmax; this one lets a
-// fused launch run its append while the CTA works on keys the append does not touch.
-__device__ __forceinline__ bool tile_depends(const AttnParams& p, int j) {
-  return (j >= p.dep_a && j < p.dep_b) || j >= p.dep_c;
-}
-
-// Key tile of local index k of the piece [j0, j1).
-__device__ __forceinline__ int tile_in_piece(const AttnParams& p, int j0, int j1, int k) {
-  const int e1 = min(j1, p.dep_a);
-  const int n1 = max(0, e1 - j0);                       // [j0, dep_a)
-  if (k < n1) return j0 + k;
-  k -= n1;
-  const int b2 = max(j0, p.dep_b), e2 = min(j1, p.dep_c);
-  const int n2 = max(0, e2 - b2);                       // [dep_b, dep_c)
-  if (k < n2) return b2 + k;
-  k -= n2;
-  const int b3 = max(j0, p.dep_a), e3 = min(j1, p.dep_b);
-  const int n3 = max(0, e3 - b3);                       // [dep_a, dep_b)
-  if (k < n3) return b3 + k;
-  return max(j0, p.dep_c) + (k - n3);                   // [dep_c, j1)
-}
-
-// Work piece (unit u2, tiles [j0, j1)) that ends at step hi (exclusive) of the range.
-struct Piece {
-  int u2, j0, j1;
-  int64_t lo;  // first step of the piece
-};
-__device__ __forceinline__ Piece piece_ending_at(const AttnParams& p, int64_t s_begin,
-                                                 int64_t hi) {
-  Piece pc;
-  pc.u2 = (int)((hi - 1) / p.n_tiles);
-  pc.lo = max(s_begin, (int64_t)pc.u2 * p.n_tiles);
-  pc.j0 = (int)(pc.lo - (int64_t)pc.u2 * p.n_tiles);
-  pc.j1 = (int)(hi - (int64_t)pc.u2 * p.n_tiles);
-  return pc;
-}
-
-// (unit, key tile) of the idx-th step the CTA processes (idx < s_end - s_begin).
-__device__ __forceinline__ void step_at(const AttnParams& p, int64_t s_begin, int64_t s_end,
-                                        int64_t idx, int* u2, int* j) {
-  int64_t hi = s_end;
-  for (;;) {
-    const Piece pc = piece_ending_at(p, s_begin, hi);
-    const int64_t n = hi - pc.lo;
-    if (idx < n) {
-      *u2 = pc.u2;
-      *j = tile_in_piece(p, pc.j0, pc.j1, (int)idx);
-      return;
-    }
-    idx -= n;
-    hi = pc.lo;
   }
 }
 
@@ -401,50 +335,15 @@ struct PageBatch {
   int page, len;
 };
 
-__device__ __forceinline__ PageBatch fetch_pages(const AttnParams& p, int64_t s_begin,
-                                                 int64_t s_end, int64_t i0, int fallback,
-                                                 int lane) {
+__device__ __forceinline__ PageBatch fetch_pages(const AttnParams& p, int64_t s0, int64_t s_end,
+                                                 int fallback, int lane) {
   PageBatch b{fallback, 0};
-  const int64_t i = i0 + lane / kPagesPerTile;  // step index within the CTA's range
-  if (lane < kBatchTiles * kPagesPerTile && i < s_end - s_begin) {
-    int u2, j;
-    step_at(p, s_begin, s_end, i, &u2, &j);
+  const int64_t s = s0 + lane / kPagesPerTile;
+  if (lane < kBatchTiles * kPagesPerTile && s < s_end) {
+    const int j = (int)(s % p.n_tiles);
     resolve_page(p, j * kPagesPerTile + lane % kPagesPerTile, fallback, &b.page, &b.len);
   }
   return b;
-}
-
-// Does any of the steps [i0, i0 + n) read pages that the fused append writes?
-__device__ __forceinline__ bool steps_depend(const AttnParams& p, int64_t s_begin, int64_t s_end,
-                                             int64_t i0, int n) {
-  for (int k = 0; k < n && i0 + k < s_end - s_begin; ++k) {
-    int u2, j;
-    step_at(p, s_begin, s_end, i0 + k, &u2, &j);
-    if (tile_depends(p, j)) return true;
-  }
-  return false;
-}
-
-// Waits (bounded) until the fused append's items are all done; then its generic-proxy writes
-// (pages, page-table row, trajectory list) are visible to this thread's TMA copies.
-__device__ __forceinline__ bool wait_append(const AttnParams& p, Shared& sh) {
-  const uint64_t t0 = global_timer();
-  for (uint32_t i = 0;; ++i) {
-    unsigned long long d;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(d) : "l"(p.done) : "memory");
-    if ((int64_t)d >= p.append_items) break;
-    if ((i & 15u) == 15u) {
-      if (sh.abort_flag) return false;
-      if (global_timer() - t0 > p.wait_ns) {
-        sh.abort_flag = 1;
-        atomicOr(p.err, GCA_DEVERR_WAIT_TIMEOUT);
-        return false;
-      }
-    }
-    __nanosleep(64);
-  }
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-  return true;
 }
 
 // ------------------------------------------------------------------------- roles
@@ -455,42 +354,28 @@ __device__ __forceinline__ void tma_producer(const CUtensorMap* tm_k, const CUte
                                              const AttnParams& p, Shared& sh, uint8_t* k_smem,
                                              uint8_t* v_smem, int64_t s_begin, int64_t s_end) {
   const int lane = threadIdx.x & 31;
-  // page of the masked slots past a work unit's last logical page: any page will do (its
-  // contents are finite: the pool is zeroed at creation and only ever holds appended keys)
-  const int fallback = 0;
+  int fallback = 0, flen = 0;
+  resolve_page(p, 0, 0, &fallback, &flen);
   uint32_t it = 0;
   uint32_t issued_k = 0, issued_v = 0;  // tiles whose copies were issued (a prefix of it)
   bool ok = true;
   // test hook: CTA 0 never issues the copies of its first tile, so the MMA issuer's wait for
   // them runs out (nothing is in flight for that tile at any time)
   const bool withhold_first = p.withhold != 0 && blockIdx.x == 0;
-  // In a fused launch, the page ids and contents of dependent key tiles are read only after
-  // the append is done: the wait comes before the first page batch that holds such a tile.
-  bool appended = p.fused == 0;
-  auto fetch = [&](int64_t i0, PageBatch* b) -> bool {
-    if (!appended && steps_depend(p, s_begin, s_end, i0, kBatchTiles)) {
-      if (!__all_sync(0xffffffffu, wait_append(p, sh))) return false;
-      appended = true;
-    }
-    *b = fetch_pages(p, s_begin, s_end, i0, fallback, lane);
-    return true;
-  };
-  PageBatch cur, nxt;
-  ok = fetch(0, &cur) && fetch(kBatchTiles, &nxt);
-  for (int64_t hi = s_end; hi > s_begin && ok;) {
-    const Piece pc = piece_ending_at(p, s_begin, hi);
-    const int h = pc.u2 / p.n_pairs;
-    const int n = pc.j1 - pc.j0;
-    for (int k = 0; k < n; ++k, ++it) {
+  PageBatch cur = fetch_pages(p, s_begin, s_end, fallback, lane);
+  PageBatch nxt = fetch_pages(p, s_begin + kBatchTiles, s_end, fallback, lane);
+  for (int64_t s = s_begin; s < s_end && ok;) {
+    const int u2 = (int)(s / p.n_tiles);
+    const int64_t seg_end = min(s_end, (int64_t)(u2 + 1) * p.n_tiles);
+    const int h = u2 / p.n_pairs;
+    const int j_end = (int)(seg_end - (int64_t)u2 * p.n_tiles);
+    for (int j = (int)(s - (int64_t)u2 * p.n_tiles); j < j_end; ++j, ++it) {
       const int st = it % kStages;
       const uint32_t use = it / kStages;
       const int kb = (int)(it % kBatchTiles);
       if (kb == 0 && it > 0) {
         cur = nxt;
-        if (!fetch((int64_t)it + kBatchTiles, &nxt)) {
-          ok = false;
-          break;
-        }
+        nxt = fetch_pages(p, s_begin + it + kBatchTiles, s_end, fallback, lane);
       }
       int page = __shfl_sync(0xffffffffu, cur.page, kb * kPagesPerTile + lane % kPagesPerTile);
       int len = __shfl_sync(0xffffffffu, cur.len, kb * kPagesPerTile + lane % kPagesPerTile);
@@ -501,8 +386,8 @@ __device__ __forceinline__ void tma_producer(const CUtensorMap* tm_k, const CUte
       }
       uint64_t lens = 0;
 #pragma unroll
-      for (int q = 0; q < kPagesPerTile; ++q) {
-        lens |= (uint64_t)(uint32_t)__shfl_sync(0xffffffffu, len, q) << (8 * q);
+      for (int k = 0; k < kPagesPerTile; ++k) {
+        lens |= (uint64_t)(uint32_t)__shfl_sync(0xffffffffu, len, k) << (8 * k);
       }
       const int row = (page * p.H + h) * kPageSize;
       if (use > 0 && !warp_wait<false>(&sh.k_empty[st], (use - 1) & 1u, &sh, p)) {
@@ -541,7 +426,7 @@ __device__ __forceinline__ void tma_producer(const CUtensorMap* tm_k, const CUte
       }
       issued_v = it + 1;
     }
-    hi = pc.lo;
+    s = seg_end;
   }
   // Drain: wait until the copies issued last have landed before the CTA can exit (a stage is
   // reissued only after its previous copy was consumed, so only the last kStages can be live).
@@ -563,9 +448,10 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, Shared& sh, uint
   const uint64_t q_desc = sw128_desc(smem_addr(q_smem + qq * kQTileBytes), 16, 1024);
   uint32_t it = 0, seg = 0;
   bool ok = true;
-  for (int64_t hi = s_end; hi > s_begin && ok; ++seg) {
-    const Piece pc = piece_ending_at(p, s_begin, hi);
-    const int n = pc.j1 - pc.j0;
+  for (int64_t s = s_begin; s < s_end && ok; ++seg) {
+    const int u2 = (int)(s / p.n_tiles);
+    const int64_t seg_end = min(s_end, (int64_t)(u2 + 1) * p.n_tiles);
+    const int n = (int)(seg_end - s);
     if (!wait_phase<true>(&sh.q_full[qq], seg & 1u, &sh, p)) break;
     tc_fence_after();
     for (int i = 0; i <= n; ++i) {
@@ -603,7 +489,7 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, Shared& sh, uint
       }
     }
     it += n;
-    hi = pc.lo;
+    s = seg_end;
   }
   // Teardown: TMEM may be freed only once every MMA issued here has completed.
   mma_commit(&sh.mma_drain[qq]);
@@ -628,18 +514,18 @@ __device__ __forceinline__ void softmax_group(const AttnParams& p, Shared& sh, u
   uint64_t* const my_turn = &sh.turn[qq];
   uint64_t* const their_turn = &sh.turn[qq ^ 1];
   if (qq == 1) mbar_arrive(their_turn);
-  for (int64_t hi = s_end; hi > s_begin && ok;) {
-    const Piece pc = piece_ending_at(p, s_begin, hi);
-    const int u2 = pc.u2, j0 = pc.j0, j1 = pc.j1;
+  for (int64_t s = s_begin; s < s_end && ok;) {
+    const int u2 = (int)(s / p.n_tiles);
+    const int64_t seg_end = min(s_end, (int64_t)(u2 + 1) * p.n_tiles);
+    const int j0 = (int)(s - (int64_t)u2 * p.n_tiles);
+    const int j1 = (int)(seg_end - (int64_t)u2 * p.n_tiles);
     const int h = u2 / p.n_pairs;
     const int qt = (u2 % p.n_pairs) * kQPerCta + qq;
     const int qi = qt * kTileQ + r;
 
     // Q row -> shared memory, 128-byte swizzle (16-byte chunk c of row r at c ^ (r % 8)),
     // and its squared norm. The previous segment's MMAs that read this tile have completed
-    // (its epilogue waited for the last P V, issued after every S of the segment). A fused
-    // launch reads the raw queries and applies the frame's 3D RoPE here, with the append's
-    // arithmetic (bit-identical to the q_rot an append writes).
+    // (its epilogue waited for the last P V, issued after every S of the segment).
     float q2 = 0.f;
     {
       const bool valid = qt < p.n_qt && qi < p.T;
@@ -648,18 +534,6 @@ __device__ __forceinline__ void softmax_group(const AttnParams& p, Shared& sh, u
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint4 v = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-        if (p.fused && valid) {
-          float2 cs[4];
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            cs[w] = append_item::rope_cs(p.ap.rope_t, p.ap.rope_tok, p.ap.nt, p.ap.nyx,
-                                         p.ap.rope_frame, qi, 4 * c + w);
-          }
-          v.x = append_item::rotate_word(v.x, cs[0]);
-          v.y = append_item::rotate_word(v.y, cs[1]);
-          v.z = append_item::rotate_word(v.z, cs[2]);
-          v.w = append_item::rotate_word(v.w, cs[3]);
-        }
         *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = v;
         const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -680,9 +554,7 @@ __device__ __forceinline__ void softmax_group(const AttnParams& p, Shared& sh, u
 
     float m_run = -INFINITY;  // running row max, log2 units (scaled)
     float l_run = 0.f;        // running row sum relative to m_run
-    for (int k = 0; k < j1 - j0; ++k, ++it) {
-      // keys the fused append is writing: kmax may not cover them yet, so the exact max runs
-      const bool dep = p.fused && tile_depends(p, tile_in_piece(p, j0, j1, k));
+    for (int j = j0; j < j1; ++j, ++it) {
       const uint32_t b = it & 1u;
       if (!warp_wait<false>(&sh.s_full[qq][b], (it >> 1) & 1u, &sh, p)) { ok = false; break; }
       if (!warp_wait<false>(&sh.lens_full[it % kLensRing], (it / kLensRing) & 1u, &sh, p)) {
@@ -711,7 +583,7 @@ __device__ __forceinline__ void softmax_group(const AttnParams& p, Shared& sh, u
         }
       }
       float m_new = m_run, alpha = 1.f;
-      if (dep || !(score_bound <= m_run + kRescaleThreshold)) {
+      if (!(score_bound <= m_run + kRescaleThreshold)) {
         // row max: 8 independent chains of 3-input max
         float mx[8];
 #pragma unroll
@@ -730,13 +602,13 @@ __device__ __forceinline__ void softmax_group(const AttnParams& p, Shared& sh, u
         if (tile_max > m_run + kRescaleThreshold) {
           m_new = tile_max;
           alpha = ex2(m_run - m_new);
-          n_rescale += k > 0 ? 1u : 0u;
+          n_rescale += j > j0 ? 1u : 0u;
         }
-        n_exact += k > 0 ? 1u : 0u;
+        n_exact += j > j0 ? 1u : 0u;
       }
       // Lazy rescale of O (rare): O += P(j-1) V must have completed first; P(j) V is issued
       // only after this thread's p_full arrival below.
-      if (k > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      if (j > j0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         const uint32_t pb = (it - 1) & 1u;
         if (!warp_wait<false>(&sh.pv_done[qq][pb], ((it - 1) >> 1) & 1u, &sh, p)) {
           ok = false;
@@ -825,53 +697,13 @@ __device__ __forceinline__ void softmax_group(const AttnParams& p, Shared& sh, u
         p.part_ml[slot * kTileQ + r] = make_float2(m_run, l_run);
       }
     }
-    hi = pc.lo;
+    s = seg_end;
   }
   // one atomic per warp and counter, at the end
   const uint32_t we = __reduce_add_sync(0xffffffffu, n_exact);
   const uint32_t wr = __reduce_add_sync(0xffffffffu, n_rescale);
   if (lane == 0 && we != 0u) atomicAdd(&p.counters[0], (unsigned long long)we);
   if (lane == 0 && wr != 0u) atomicAdd(&p.counters[1], (unsigned long long)wr);
-}
-
-// Warp 11 of a fused launch: the frame's append (RoPE + paged scatter of K and V, eviction).
-// Items are claimed kClaimItems at a time from the launch's claim counter, the next claim taken
-// while the current items run, so every CTA that runs takes part and none waits for a CTA that
-// has not started: this warp never waits for anything but its own memory operations, so the
-// append completes however many CTAs are resident. Item order: token chunks (chunk fastest,
-// then head, then slot), then the eviction items. Claims are multiples of 8 items, so the 8
-// chunks of one (token, head) sit in 8 consecutive lanes, as the per-item code expects.
-__device__ __forceinline__ void append_warp(const AttnParams& p) {
-  const int lane = threadIdx.x & 31;
-  const AppendParams& a = p.ap;
-  const int64_t n_tok = (int64_t)a.ppf * kPageSize * a.H * 8;
-  const int64_t total = p.append_items;
-  unsigned long long claim = 0;
-  if (lane == 0) claim = atomicAdd(p.claim, (unsigned long long)kClaimItems);
-  claim = __shfl_sync(0xffffffffu, claim, 0);
-  int64_t mine = 0;
-  while ((int64_t)claim < total) {
-    unsigned long long next = 0;
-    if (lane == 0) next = atomicAdd(p.claim, (unsigned long long)kClaimItems);
-#pragma unroll
-    for (int q = 0; q < kClaimItems / 32; ++q) {
-      const int64_t idx = (int64_t)claim + 32 * q + lane;
-      if (idx < n_tok) {
-        const int64_t th = idx >> 3;
-        append_item::token_chunk<false>(a, (int)(th / a.H), (int)(th % a.H), (int)(idx & 7));
-      } else if (idx < total) {
-        append_item::aux(a, idx - n_tok);
-      }
-    }
-    mine += min((int64_t)kClaimItems, total - (int64_t)claim);
-    claim = __shfl_sync(0xffffffffu, next, 0);
-  }
-  // every lane's stores, then the count: a reader that sees the count sees the stores
-  __syncwarp();
-  if (lane == 0 && mine > 0) {
-    __threadfence();
-    atomicAdd(p.done, (unsigned long long)mine);
-  }
 }
 
 // ------------------------------------------------------------------------- kernel
@@ -926,23 +758,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Everything above is local (barriers, TMEM); from here on the kernel reads the page table,
   // Q, K and V that earlier work in the stream wrote.
   pdl_wait();
-  // The previous fused launch has completed (the stream's order and the wait above): its
-  // counter pair is free and becomes the next fused launch's, zeroed here.
-  if (p.fused && blockIdx.x == 0 && threadIdx.x == 0) {
-    p.next_counters[0] = 0ull;
-    p.next_counters[1] = 0ull;
-  }
 
   // A cache whose sticky error word is set gets no further work: every role sees an empty step
-  // range and the CTA goes straight to its teardown (a fused launch then appends nothing).
+  // range and the CTA goes straight to its teardown.
   const bool dead = *reinterpret_cast<volatile uint32_t*>(p.err) != 0u;
   const int64_t s_begin = (int64_t)blockIdx.x * p.total / p.grid;
   const int64_t s_end = dead ? s_begin : (int64_t)(blockIdx.x + 1) * p.total / p.grid;
 
   if (warp == kWarpTma) {
     tma_producer(&tm_k, &tm_v, p, sh, k_smem, v_smem, s_begin, s_end);
-  } else if (warp == kWarpAppend) {
-    if (p.fused && !dead) append_warp(p);
   } else if (warp == kWarpMma0 || warp == kWarpMma0 + 1) {
     if ((threadIdx.x & 31) == 0) {
       mma_issuer(p, sh, tmem, q_smem, k_smem, v_smem, warp - kWarpMma0, s_begin, s_end);

@@ -89,7 +89,6 @@ struct Layout {
   size_t err;                // uint32 sticky device error word
   size_t kmax;               // float [H] (as uint32 bits): max squared key norm ever appended
   size_t counters;           // uint64 [4]: attention branch counters (gca_read_attend_counters)
-  size_t step_counters;      // uint64 [2][2]: claim / done counters of fused launches (by parity)
   size_t part_o;             // float [part_slots][128][64]
   size_t part_ml;            // float2 [part_slots][128]
   size_t total;
@@ -196,17 +195,6 @@ struct AttnParams {
   uint64_t wait_ns;      // bound of every pipeline wait (a wait that runs out sets
                          // GCA_DEVERR_WAIT_TIMEOUT and the CTA winds down)
   int32_t withhold;      // test hook: 1 = CTA 0 never issues the copies of its first key tile
-  // Fused launch (gca_append_attend): the frame's append runs inside the attention launch. Its
-  // items (token chunks, then eviction items) are claimed by one warp per CTA; key tiles
-  // [dep_a, dep_b) and [dep_c, n_tiles) read pages that the append writes and are loaded only
-  // once `done` has counted every item. Without fusion dep_a = dep_b = dep_c = n_tiles.
-  int32_t fused;
-  int32_t dep_a, dep_b, dep_c;
-  int64_t append_items;
-  unsigned long long* claim;          // this launch's claim counter (zeroed beforehand)
-  unsigned long long* done;           // this launch's completed-item counter (zeroed beforehand)
-  unsigned long long* next_counters;  // claim and done of the next fused launch: zeroed here
-  AppendParams ap;                    // the append (q_rot unused: queries rotate on load)
 };
 
 // Launchers (return cudaGetLastError() of the launch).
@@ -260,7 +248,6 @@ struct gca_cache {
   uint32_t dev_err;
   uint64_t wait_ns;        // attention wait bound (gca_set_wait_limit)
   int32_t withhold_next;   // test hook armed for the next attention launch
-  int64_t fused_launches;  // fused launches since create / reset (selects the counter pair)
   cudaEvent_t split_event; // measurement hook: recorded between attention and combine launches
   CUtensorMap tm_k;
   CUtensorMap tm_v;

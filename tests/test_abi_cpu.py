@@ -106,7 +106,6 @@ def test_create_rejects_bad_arguments_before_touching_cuda(L):
     assert L.gca_append_frame_ex(None, 0, 0, 0, 1, 1, 1, 1, None) == -1
     assert L.gca_rollback_last_frame(None, 0, None) == -1
     assert L.gca_attend_prefill(None, 1, 1, 1, None) == -1
-    assert L.gca_append_attend(None, 0, 16, 16, 16, 16, None) == -1
     # batched append: empty or oversized batch, null arrays, null cache
     VP, I64 = ctypes.c_void_p, ctypes.c_int64
     one = (VP * 1)(1)
@@ -138,7 +137,6 @@ def test_binding_routes_each_call_to_its_entry_point(L):
     assert where(cache.append_frame, 0, x, x, x, x, stream=0, rope_frame=3) == \
         "gca_append_frame_ex"
     assert where(cache.attend, 0, x, x, stream=0) == "gca_attend"
-    assert where(cache.append_attend, 0, x, x, x, x, stream=0) == "gca_append_attend"
     assert where(cache.attend_prefill, 2, x, x, stream=0) == "gca_attend_prefill"
     assert where(cache.rollback, 0) == "gca_rollback_last_frame"
     assert where(cache.reset, stream=0) == "gca_reset"
