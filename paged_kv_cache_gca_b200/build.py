@@ -35,7 +35,7 @@ def build_command(verbose: bool = False, out: str | None = None) -> list[str]:
 
 def build(verbose: bool = False, force: bool = False) -> str:
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
-    deps = srcs + [os.path.join(CSRC, "gca_internal.h"), os.path.join(CSRC, "gca_append_item.cuh"),
+    deps = srcs + [os.path.join(CSRC, "gca_internal.h"),
                    os.path.join(os.path.dirname(HERE), "include", "gca.h")]
     if not force and os.path.exists(LIB):
         lib_t = os.path.getmtime(LIB)

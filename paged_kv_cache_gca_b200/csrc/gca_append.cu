@@ -1,8 +1,7 @@
 // Append-side kernels of the GCA paged KV cache (sm_100a).
 //
-// append_kernel does one frame's whole append step in a single launch (the per-item code and
-// its description are in gca_append_item.cuh), following the order of the pages' streaming
-// block ("How the Geometric Context Transformer Enables Streaming 3D
+// gca_append_kernel does one frame's whole append step in a single launch, following the order
+// of the pages' streaming block ("How the Geometric Context Transformer Enables Streaming 3D
 // Reconstruction in LingBot-Map", FlashInferBlock: append_frame, then evict_frames):
 //   a1  the frame's pages are popped from the FIFO free list (ring positions free_head ..
 //       free_head+ppf-1) and written to its page-table row; slot_map[i] = page*16 + i%16;
@@ -19,7 +18,7 @@
 // (A+W)*ppf pages are in use.
 #include <cuda_bf16.h>
 
-#include "gca_append_item.cuh"
+#include "gca_internal.h"
 
 namespace gca {
 
@@ -27,7 +26,7 @@ namespace {
 
 constexpr int kThreads = 256;
 
-using append_item::set_err;
+__device__ __forceinline__ void set_err(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
 
 // ------------------------------------------------------------------------------- init
 
@@ -103,6 +102,25 @@ __global__ void reset_kernel(int32_t* free_ring, const int32_t* init_free, uint3
 
 // ------------------------------------------------------------------------------- append
 
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+
+// Rotates the pair held in one 32-bit word (element 2j in the low half, 2j+1 in the high half).
+__device__ __forceinline__ uint32_t rotate_word(uint32_t w, float2 cs) {
+  const float a = bf_lo(w), b = bf_hi(w);
+  const float ra = fmaf(a, cs.x, -b * cs.y);
+  const float rb = fmaf(a, cs.y, b * cs.x);
+  return pack_bf2(ra, rb);
+}
+
+__device__ __forceinline__ int wrap(int pos, int n) { return pos >= n ? pos - n : pos; }
+
+
 // Block bx of one cache's append. Token part: block (8 chunks, H heads, tok_per_block tokens);
 // one thread = one 16-byte chunk (8 dims) of one (token, head). Auxiliary part (blocks after
 // n_tok_blocks): eviction copies, zero fill of a fresh trajectory page, free-list pushes,
@@ -113,16 +131,138 @@ __device__ __forceinline__ void append_block(const AppendParams& p, const int bx
   // register pressure): every page id is range-checked before any write, so it stays in
   // bounds, and the attention and combine kernels, which do test the word, write no output.
   if (bx < p.n_tok_blocks) {
+    // ---- a1 + a2
+    const int c = threadIdx.x;
+    const int h = threadIdx.y;
     const int i = bx * p.tok_per_block + threadIdx.z;
     if (i >= p.ppf * kPageSize) return;
-    // the 8 chunks of one (token, head) are 8 consecutive lanes (threads are linearised x first)
-    append_item::token_chunk<true>(p, i, threadIdx.y, threadIdx.x);
+    const int page = p.free_ring[wrap(p.head_pos + i / kPageSize, p.num_pages)];
+    if (page < 0 || page >= p.num_pages) {
+      set_err(p.err, GCA_DEVERR_PAGE_RANGE);
+      return;
+    }
+    const int slot = i % kPageSize;
+    const int64_t dst = (((int64_t)page * H + h) * kPageSize + slot) * 8 + c;
+    if (i >= p.T) {  // padding slot of the frame's last page
+      p.k_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
+      p.v_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
+      return;
+    }
+    const int64_t src = ((int64_t)i * H + h) * 8 + c;
+    const uint4 qv = p.q[src];
+    const uint4 kv = p.k[src];
+    const uint4 vv = p.v[src];
+    float2 cs[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int j = 4 * c + w;  // pair index within the head
+      cs[w] = j < p.nt ? p.rope_t[p.rope_frame * p.nt + j]
+                     : p.rope_tok[(int64_t)i * p.nyx + (j - p.nt)];
+    }
+    uint4 qr, kr;
+    qr.x = rotate_word(qv.x, cs[0]);
+    qr.y = rotate_word(qv.y, cs[1]);
+    qr.z = rotate_word(qv.z, cs[2]);
+    qr.w = rotate_word(qv.w, cs[3]);
+    kr.x = rotate_word(kv.x, cs[0]);
+    kr.y = rotate_word(kv.y, cs[1]);
+    kr.z = rotate_word(kv.z, cs[2]);
+    kr.w = rotate_word(kv.w, cs[3]);
+    if (h == 0 && c == 0) {
+      p.slot_map[i] = page * kPageSize + slot;
+      if (slot == 0) p.frame_pages[p.t * p.ppf + i / kPageSize] = page;
+    }
+    p.q_rot[src] = qr;
+    p.k_pool[dst] = kr;
+    p.v_pool[dst] = vv;
+    // The stored key's squared norm raises the head's running maximum: the attention bounds
+    // every score of a row by |q| * max|k| and skips its row max while that bound is below
+    // the running max + 2^8. Computed after the stores, when the q and v registers are free.
+    {
+      float ss = 0.f;
+      const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float a = bf_lo(kw[w]), b = bf_hi(kw[w]);
+        ss = fmaf(a, a, fmaf(b, b, ss));
+      }
+      // the 8 chunks of one (token, head) are 8 consecutive lanes
+      const unsigned lane = (threadIdx.x + 8u * (threadIdx.y + (unsigned)H * threadIdx.z)) & 31u;
+      const unsigned group = 0xffu << (lane & 24u);
+      ss += __shfl_xor_sync(group, ss, 1);
+      ss += __shfl_xor_sync(group, ss, 2);
+      ss += __shfl_xor_sync(group, ss, 4);
+      if (c == 0 && ss > __uint_as_float(p.kmax[h])) atomicMax(&p.kmax[h], __float_as_uint(ss));
+    }
     return;
   }
+
   const int block_threads = 8 * H * p.tok_per_block;
   const int lin = threadIdx.x + 8 * (threadIdx.y + H * threadIdx.z);
   const int64_t idx = (int64_t)(bx - p.n_tok_blocks) * block_threads + lin;
-  if (idx < p.n_aux_items) append_item::aux(p, idx);
+  if (idx >= p.n_aux_items) return;
+  const int64_t e_ev = p.n_evict_items;
+  const int64_t e_zero = e_ev + p.n_zero_items;
+  const int64_t e_push = e_zero + p.n_push_items;
+  const int first_new = wrap(p.head_pos + p.ppf, p.num_pages);  // first trajectory pop
+
+  if (idx < e_ev) {
+    // ---- a3: copy kept token j of the evicted frame to trajectory position traj_len + j
+    const int c = (int)(idx & 7);
+    const int64_t th = idx >> 3;
+    const int h = (int)(th % H);
+    const int j = (int)(th / H);
+    const int tok = p.kept[j];
+    const int src_page = p.frame_pages[(int64_t)p.evict_frame * p.ppf + tok / kPageSize];
+    const int64_t pos = p.traj_len + j;
+    const int64_t tp = pos / kPageSize;
+    const int dst_page =
+        tp < p.traj_pages_before
+            ? p.traj_pages[tp]
+            : p.free_ring[wrap(first_new + (int)(tp - p.traj_pages_before), p.num_pages)];
+    if (src_page < 0 || src_page >= p.num_pages || dst_page < 0 || dst_page >= p.num_pages) {
+      set_err(p.err, GCA_DEVERR_PAGE_RANGE);
+      return;
+    }
+    const int64_t src = (((int64_t)src_page * H + h) * kPageSize + tok % kPageSize) * 8 + c;
+    const int64_t dst = (((int64_t)dst_page * H + h) * kPageSize + pos % kPageSize) * 8 + c;
+    p.k_pool[dst] = p.k_pool[src];
+    p.v_pool[dst] = p.v_pool[src];
+    return;
+  }
+
+  if (idx < e_zero) {
+    // ---- zero the slots of the last new trajectory page that this step leaves empty
+    const int64_t r = idx - e_ev;
+    const int c = (int)(r & 7);
+    const int64_t th = r >> 3;
+    const int h = (int)(th % H);
+    const int z = (int)(th / H);
+    const int64_t pos = p.traj_len + p.K + z;
+    const int64_t tp = pos / kPageSize;
+    const int page =
+        p.free_ring[wrap(first_new + (int)(tp - p.traj_pages_before), p.num_pages)];
+    if (page < 0 || page >= p.num_pages) {
+      set_err(p.err, GCA_DEVERR_PAGE_RANGE);
+      return;
+    }
+    const int64_t dst = (((int64_t)page * H + h) * kPageSize + pos % kPageSize) * 8 + c;
+    p.k_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
+    p.v_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+
+  if (idx < e_push) {
+    // ---- push the evicted frame's pages to the free-list tail, in row order
+    const int k = (int)(idx - e_zero);
+    p.free_ring[wrap(p.tail_pos + k, p.num_pages)] =
+        p.frame_pages[(int64_t)p.evict_frame * p.ppf + k];
+    return;
+  }
+
+  // ---- record the trajectory pages popped by this step
+  const int k = (int)(idx - e_push);
+  p.traj_pages[p.traj_pages_before + k] = p.free_ring[wrap(first_new + k, p.num_pages)];
 }
 
 // At most 512 threads (8 chunks x 64 heads) and 32 registers: 8 blocks of 256 threads per SM
@@ -130,26 +270,9 @@ __device__ __forceinline__ void append_block(const AppendParams& p, const int bx
 // slower).
 #define GCA_APPEND_BOUNDS __launch_bounds__(512, 4)
 
-// One frame's append: warp w of the grid takes token items [128 w, 128 w + 128), four per lane
-// with their loads in flight together (a single 12 MB frame is one short wave, so memory-level
-// parallelism per thread, not occupancy, bounds it); the warps after the token items take the
-// eviction items, one per lane.
-constexpr int kAppendWarpsPerBlock = 8;
-constexpr int kItemsPerWarp = 128;
-
-__global__ void __launch_bounds__(32 * kAppendWarpsPerBlock)
-    append_kernel(const AppendParams p) {
+__global__ void GCA_APPEND_BOUNDS append_kernel(const AppendParams p) {
   pdl_wait();  // inputs, pages and the free ring may come from earlier work in the stream
-  const int lane = threadIdx.x & 31;
-  const int64_t warp = (int64_t)blockIdx.x * kAppendWarpsPerBlock + (threadIdx.x >> 5);
-  const int64_t n_tok = (int64_t)p.ppf * kPageSize * p.H * 8;
-  const int64_t tok_warps = n_tok / kItemsPerWarp;
-  if (warp < tok_warps) {
-    append_item::token_chunks4<true>(p, warp * kItemsPerWarp, lane);
-  } else {
-    const int64_t idx = (warp - tok_warps) * 32 + lane;
-    if (idx < p.n_aux_items) append_item::aux(p, idx);
-  }
+  append_block(p, (int)blockIdx.x);
   pdl_launch_dependents();
 }
 
@@ -185,12 +308,8 @@ cudaError_t launch_reset(int32_t* free_ring, const int32_t* init_free, uint32_t*
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
-  // token items: ppf * 16 slots x H heads x 8 chunks, a multiple of 128 since 16 * 8 = 128
-  const int64_t n_tok = (int64_t)p.ppf * kPageSize * p.H * 8;
-  const int64_t warps = n_tok / kItemsPerWarp + (p.n_aux_items + 31) / 32;
-  const int64_t blocks = (warps + kAppendWarpsPerBlock - 1) / kAppendWarpsPerBlock;
-  return launch_dependent(append_kernel, dim3((unsigned)blocks),
-                          dim3(32 * kAppendWarpsPerBlock), 0, s, p);
+  const dim3 block(8, p.H, p.tok_per_block);
+  return launch_dependent(append_kernel, dim3((unsigned)p.n_blocks), block, 0, s, p);
 }
 
 cudaError_t launch_append_batch(const AppendBatch& b, cudaStream_t s) {
