@@ -208,7 +208,10 @@ gca_status gca_append_frames(gca_cache* const* caches, int32_t n, const int64_t*
  * trajectory keys visible at frame frame_idx (which must be the last appended frame).
  * q_rot: device bf16 [T][H][D] from gca_append_frame; out: device bf16 [T][H][D], not
  * overlapping q_rot (GCA_ERR_INVALID_ARG: CTAs still read queries while others write rows).
- * One tcgen05 attention launch, plus one combine launch when the key range is split. */
+ * One tcgen05 attention launch, plus one combine launch when the key range is split. A frame
+ * of at most 4 tokens (the causal camera head's cache: one camera token per frame) attends on
+ * CUDA cores instead, in one launch: per head a cluster of up to 8 CTAs splits the key pages
+ * and merges in on-chip shared memory (gca_attend_info: launches 1, grid = splits * H). */
 gca_status gca_attend(gca_cache* cache, int64_t frame_idx, const void* q_rot, void* out,
                       void* stream);
 
@@ -219,7 +222,8 @@ gca_status gca_attend(gca_cache* cache, int64_t frame_idx, const void* q_rot, vo
  * Streaming Inference API, FAQ on scale frames). q_rot: device bf16 [n*T][H][D], the q_rot
  * outputs of the n appends back to back (frame-major); out: device bf16 [n*T][H][D], not
  * overlapping q_rot (GCA_ERR_INVALID_ARG). One
- * attention launch (+ one combine launch when split). GCA_ERR_INVALID_ARG unless
+ * attention launch (+ one combine launch when split; n*T <= 4 query rows: the one-launch CUDA-
+ * core path of gca_attend). GCA_ERR_INVALID_ARG unless
  * 1 <= n <= anchor_frames; GCA_ERR_FRAME_ORDER unless exactly n frames are appended (and no
  * transient frame is pending). */
 gca_status gca_attend_prefill(gca_cache* cache, int32_t n, const void* q_rot, void* out,
@@ -241,6 +245,8 @@ gca_status gca_attend_prefill(gca_cache* cache, int32_t n, const void* q_rot, vo
  * events). The array holds 496 partial records of 128 query rows; a launch over num_heads *
  * ceil(T / 256) query-tile pairs needs two per pair and two per CTA, so this returns
  * GCA_ERR_UNSUPPORTED when num_heads * ceil(T / 256) >= 248; other errors as gca_attend.
+ * A frame of at most 4 tokens takes gca_attend's CUDA-core path, which needs no scratch (and
+ * does not touch the array).
  * The web pages have no counterpart of this entry point; it is an addition of this library. */
 gca_status gca_attend_noalloc(gca_cache* cache, int64_t frame_idx, const void* q_rot, void* out,
                               void* stream);

@@ -11,7 +11,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libgca.so")
-SOURCES = ["gca_api.cu", "gca_append.cu", "gca_attn.cu", "gca_combine.cu", "gca_noalloc.cu"]
+SOURCES = ["gca_api.cu", "gca_append.cu", "gca_attn.cu", "gca_combine.cu", "gca_decode.cu",
+           "gca_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

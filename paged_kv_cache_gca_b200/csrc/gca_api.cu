@@ -219,6 +219,35 @@ bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams
   return true;
 }
 
+// A query set of at most kDecodeMaxRows rows: one CUDA-core decode launch, the key pages of
+// each head split over a cluster of dsplit CTAs (enough CTAs to cover the SMs, at least
+// kDecodePagesPerSplit pages each, at most kDecodeMaxSplit).
+gca_status enqueue_decode(gca_cache* c, int64_t t, int64_t visible_keys, AttnParams* p,
+                          cudaStream_t s) {
+  constexpr int kDecodePagesPerSplit = 8;
+  const int64_t H = c->cfg.num_heads;
+  int64_t S = (2 * (int64_t)c->sms + H - 1) / H;
+  S = std::min<int64_t>(S, (p->n_lp + kDecodePagesPerSplit - 1) / kDecodePagesPerSplit);
+  S = std::min<int64_t>(S, kDecodeMaxSplit);
+  S = std::max<int64_t>(S, 1);
+  p->k_pool = reinterpret_cast<const uint4*>(c->ws + c->lay.k_pool);
+  p->v_pool = reinterpret_cast<const uint4*>(c->ws + c->lay.v_pool);
+  p->dsplit = (int32_t)S;
+  if (launch_decode(*p, s) != cudaSuccess) return GCA_ERR_CUDA;
+  c->withhold_next = 0;  // the test hook applies to the tensor-core kernel only
+  if (c->split_event && cudaEventRecord(c->split_event, s) != cudaSuccess) return GCA_ERR_CUDA;
+  gca_attend_info& inf = c->last;
+  inf.frame_idx = t;
+  inf.visible_keys = visible_keys;
+  inf.logical_pages = p->n_lp;
+  inf.kv_tiles = p->n_tiles;
+  inf.query_tiles = p->n_qt;
+  inf.grid = (int32_t)(S * H);
+  inf.split = S > 1 ? 1 : 0;
+  inf.launches = 1;
+  return GCA_OK;
+}
+
 }  // namespace gca
 
 using namespace gca;
@@ -538,6 +567,7 @@ gca_status enqueue_attention(gca_cache* c, int64_t t, int64_t q_rows, const void
   p.part_o = at<float>(c, L.part_o);
   p.part_ml = at<float2>(c, L.part_ml);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p.T <= kDecodeMaxRows) return enqueue_decode(c, t, nk, &p, s);
   if (launch_attn(c->tm_k, c->tm_v, p, s) != cudaSuccess) return GCA_ERR_CUDA;
   c->withhold_next = 0;
   if (c->split_event && cudaEventRecord(c->split_event, s) != cudaSuccess) return GCA_ERR_CUDA;

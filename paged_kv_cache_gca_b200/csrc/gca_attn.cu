@@ -306,26 +306,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major) {
 
 // ------------------------------------------------------------------------- page walk
 
-// Physical page and valid-slot count of logical page lp (anchor, window, trajectory order).
-__device__ __forceinline__ void resolve_page(const AttnParams& p, int lp, int fallback,
-                                             int* page, int* len) {
-  if (lp < p.na_pages) {
-    *page = p.frame_pages[lp];
-    *len = (lp % p.ppf == p.ppf - 1) ? p.last_len : kPageSize;
-  } else if (lp < p.na_pages + p.nw_pages) {
-    const int w = lp - p.na_pages;
-    *page = p.frame_pages[p.win_base + w];
-    *len = (w % p.ppf == p.ppf - 1) ? p.last_len : kPageSize;
-  } else if (lp < p.n_lp) {
-    const int tp = lp - p.na_pages - p.nw_pages;
-    *page = p.traj_pages[tp];
-    *len = (tp == p.n_traj_pages - 1) ? p.traj_tail_len : kPageSize;
-  } else {
-    *page = fallback;  // any visible page: finite data, fully masked
-    *len = 0;
-  }
-}
-
 // Page ids of kBatchTiles consecutive steps, fetched in one round of loads: lane l <
 // kBatchTiles * kPagesPerTile holds page l % kPagesPerTile of step s0 + l / kPagesPerTile (the
 // logical pages of a key tile do not depend on the work unit, only on the tile index).

@@ -195,6 +195,10 @@ struct AttnParams {
   uint64_t wait_ns;      // bound of every pipeline wait (a wait that runs out sets
                          // GCA_DEVERR_WAIT_TIMEOUT and the CTA winds down)
   int32_t withhold;      // test hook: 1 = CTA 0 never issues the copies of its first key tile
+  // decode kernel (query sets of at most kDecodeMaxRows rows)
+  const uint4* k_pool;   // [pages][H][16][64] bf16
+  const uint4* v_pool;
+  int32_t dsplit;        // key splits per head: one cluster of dsplit CTAs per head
 };
 
 // Launchers (return cudaGetLastError() of the launch).
@@ -208,6 +212,36 @@ cudaError_t attn_prepare(int* ctas_per_sm);  // sets kernel attributes, reports 
 cudaError_t launch_attn(const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
                         cudaStream_t s);
 cudaError_t launch_combine(const AttnParams& p, cudaStream_t s);
+cudaError_t launch_decode(const AttnParams& p, cudaStream_t s);
+// Enqueues the decode launch for a planned attention of at most kDecodeMaxRows query rows
+// (p from plan_attention, q and out set) and records the launch in c->last.
+gca_status enqueue_decode(gca_cache* c, int64_t t, int64_t visible_keys, AttnParams* p,
+                          cudaStream_t s);
+
+// Query sets of at most this many rows (the causal camera head's one camera token per frame)
+// attend on CUDA cores: a 128-row tensor-core tile would be almost all padding.
+constexpr int kDecodeMaxRows = 4;
+constexpr int kDecodeMaxSplit = 8;  // CTAs per head: a portable cluster
+
+// Physical page and valid-slot count of logical page lp (anchor, window, trajectory order).
+__device__ __forceinline__ void resolve_page(const AttnParams& p, int lp, int fallback,
+                                             int* page, int* len) {
+  if (lp < p.na_pages) {
+    *page = p.frame_pages[lp];
+    *len = (lp % p.ppf == p.ppf - 1) ? p.last_len : kPageSize;
+  } else if (lp < p.na_pages + p.nw_pages) {
+    const int w = lp - p.na_pages;
+    *page = p.frame_pages[p.win_base + w];
+    *len = (w % p.ppf == p.ppf - 1) ? p.last_len : kPageSize;
+  } else if (lp < p.n_lp) {
+    const int tp = lp - p.na_pages - p.nw_pages;
+    *page = p.traj_pages[tp];
+    *len = (tp == p.n_traj_pages - 1) ? p.traj_tail_len : kPageSize;
+  } else {
+    *page = fallback;  // any visible page: finite data, fully masked
+    *len = 0;
+  }
+}
 
 // Split bookkeeping shared by the attention and combine kernels: CTA c owns the flattened
 // (pair unit, key tile) steps [c*total/grid, (c+1)*total/grid); the CTA that holds step s is

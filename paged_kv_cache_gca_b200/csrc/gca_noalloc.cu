@@ -106,6 +106,11 @@ extern "C" gca_status gca_attend_noalloc(gca_cache* c, int64_t t, const void* q_
   bool split = false;
   int64_t nk = 0;
   if (!plan_attention(c, t, kNoallocSlots, &p, &split, &nk)) return GCA_ERR_UNSUPPORTED;
+  if (p.T <= kDecodeMaxRows) {  // the decode kernel merges its splits on chip: no scratch
+    p.q = static_cast<const uint4*>(q_rot);
+    p.out = static_cast<uint4*>(out);
+    return enqueue_decode(c, t, nk, &p, static_cast<cudaStream_t>(stream));
+  }
   void* scratch = nullptr;
   if (scratch_address(dev, &scratch) != cudaSuccess) return GCA_ERR_CUDA;
   p.q = static_cast<const uint4*>(q_rot);
