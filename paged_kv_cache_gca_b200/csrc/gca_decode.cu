@@ -28,8 +28,12 @@
 namespace gca {
 namespace {
 
-constexpr int kDecodeThreads = 256;
-constexpr int kDecodeWarps = kDecodeThreads / 32;
+// Warps per CTA. 8 keeps two to three CTAs resident per SM, so a launch of 8 splits x 32 heads
+// is one wave (16 warps hold an SM per CTA and took twice as long).
+template <int kRows>
+__host__ __device__ constexpr int decode_warps() {
+  return 8;
+}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -41,7 +45,8 @@ __device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 template <int kRows>
-__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(32 * decode_warps<kRows>()) decode_kernel(const AttnParams p) {
+  constexpr int kDecodeWarps = decode_warps<kRows>();
   namespace cg = cooperative_groups;
   pdl_wait();  // the append that wrote this frame's keys and the page table
   cg::cluster_group cluster = cg::this_cluster();
@@ -90,9 +95,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const AttnParams
 
   const int lp0 = (int)((int64_t)split * p.n_lp / n_split);
   const int lp1 = live ? (int)((int64_t)(split + 1) * p.n_lp / n_split) : lp0;
+  // the page id of the warp's next page is read while the current page is processed
+  int next_page = 0, next_len = 0;
+  if (lp0 + warp < lp1) resolve_page(p, lp0 + warp, 0, &next_page, &next_len);
   for (int lp = lp0 + warp; lp < lp1; lp += kDecodeWarps) {
-    int page = 0, len = 0;
-    resolve_page(p, lp, 0, &page, &len);
+    const int page = next_page, len = next_len;
+    if (lp + kDecodeWarps < lp1) resolve_page(p, lp + kDecodeWarps, 0, &next_page, &next_len);
     if (page < 0 || page >= p.num_pages) {  // the same for every lane of the warp
       if (lane == 0) atomicOr(p.err, GCA_DEVERR_PAGE_RANGE);
       continue;
@@ -213,17 +221,18 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const AttnParams
 
 cudaError_t launch_decode(const AttnParams& p, cudaStream_t s) {
   void (*kernel)(const AttnParams) = nullptr;
+  int warps = 0;
   switch (p.T) {
-    case 1: kernel = decode_kernel<1>; break;
-    case 2: kernel = decode_kernel<2>; break;
-    case 3: kernel = decode_kernel<3>; break;
-    case 4: kernel = decode_kernel<4>; break;
+    case 1: kernel = decode_kernel<1>; warps = decode_warps<1>(); break;
+    case 2: kernel = decode_kernel<2>; warps = decode_warps<2>(); break;
+    case 3: kernel = decode_kernel<3>; warps = decode_warps<3>(); break;
+    case 4: kernel = decode_kernel<4>; warps = decode_warps<4>(); break;
     default: return cudaErrorInvalidValue;
   }
   if (p.dsplit < 1 || p.dsplit > kDecodeMaxSplit) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.dsplit, p.H);
-  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.blockDim = dim3(32 * warps);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
