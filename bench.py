@@ -756,9 +756,10 @@ def run_e2e(args, w, cache, ring_host, device, stream, world):
     """Frames/s through the public API with inputs in pinned host memory: every frame's q, k, v
     are copied host->device and its output device->host inside the timed region. Copies move
     chunks of 8 frames on their own streams (one copy engine each way), ordered against the
-    compute stream by events, with three rotating chunk buffers each way: chunk c+1's upload and
-    chunk c-1's download overlap chunk c's compute, and the 8 frames of a chunk run with no
-    stream operation between their launches."""
+    compute stream by events, with three chunk buffers each way rotating across steps: chunk
+    c+1's upload and chunk c-1's download overlap chunk c's compute (a step's first uploads
+    overlap the previous step's last chunks), and the 8 frames of a chunk run with no stream
+    operation between their launches."""
     T, H, D = w.tokens_per_frame, w.num_heads, w.head_dim
     nframes = w.frames
     C = 8 if nframes % 8 == 0 and w.ring % 8 == 0 else 1
@@ -778,9 +779,12 @@ def run_e2e(args, w, cache, ring_host, device, stream, world):
     steps = max(1, min(args.steps, 3))
     started = [False] * nbuf      # input buffer b has been uploaded into before
     downloading = [False] * nbuf  # output buffer b has a download issued (maybe in flight)
+    # Buffers rotate over a chunk counter that runs on across steps, so the first uploads of a
+    # step go to buffers the previous step's last chunks do not hold and overlap its tail.
+    gchunk = [0]
 
-    def upload(ci):
-        b = ci % nbuf
+    def upload(ci, g):
+        b = g % nbuf
         s0 = (ci * C) % w.ring
         with torch.cuda.stream(h2d):
             if started[b]:
@@ -790,14 +794,15 @@ def run_e2e(args, w, cache, ring_host, device, stream, world):
         started[b] = True
 
     def step():
+        g0 = gchunk[0]
         cache.reset(stream=stream)
-        upload(0)
+        upload(0, g0)
         if nchunks > 1:
-            upload(1)
+            upload(1, g0 + 1)
         for ci in range(nchunks):
-            b = ci % nbuf
+            b = (g0 + ci) % nbuf
             if ci + 2 < nchunks:
-                upload(ci + 2)
+                upload(ci + 2, g0 + ci + 2)
             stream.wait_event(up[b])
             if downloading[b]:
                 stream.wait_event(down[b])  # output b's previous chunk has been downloaded
@@ -813,6 +818,7 @@ def run_e2e(args, w, cache, ring_host, device, stream, world):
                 out_host[b].copy_(out[b], non_blocking=True)
                 down[b].record(d2h)
             downloading[b] = True
+        gchunk[0] = g0 + nchunks
 
     with torch.cuda.stream(stream):
         step()
