@@ -265,12 +265,14 @@ gca_status gca_cache_destroy(gca_cache* cache);
 gca_status gca_check(gca_cache* cache);
 
 /* Synchronises the device and reads the cache's attention branch counters (for tests and
- * measurement: they show which paths of the online softmax a stream exercised). */
+ * measurement: they show which paths of the online softmax a stream exercised). The decode path
+ * of frames of at most 4 tokens keeps a plain online softmax and counts nothing. */
 gca_status gca_read_attend_counters(gca_cache* cache, gca_attend_counters* counters);
 
 /* Measurement hook: while cuda_event (a cudaEvent_t created by the caller) is set, every
  * gca_attend / gca_attend_prefill of this cache records it on the call's stream right after the
- * attention kernel's launch and before the combine's, so that events around the call split its
+ * attention kernel's launch and before the combine's (after the single launch of the decode
+ * path), so that events around the call split its
  * time between the two kernels. NULL clears it. An event between the launches stops the combine
  * from starting early (programmatic launch), so use it in a separate, instrumented pass. */
 gca_status gca_set_split_event(gca_cache* cache, void* cuda_event);
@@ -280,7 +282,8 @@ gca_status gca_set_split_event(gca_cache* cache, void* cuda_event);
  * GCA_DEVERR_WAIT_TIMEOUT in the sticky device error word; the kernel's CTAs then stop issuing
  * work, wait (bounded) for the copies and MMAs they already issued, free their tensor memory and
  * return, so the call always ends and the CUDA context stays usable. Host only; applies to
- * attention launches enqueued after the call. */
+ * attention launches enqueued after the call. The decode kernel of frames of at most 4 tokens has
+ * no pipeline waits. */
 gca_status gca_set_wait_limit(gca_cache* cache, uint64_t wait_ns);
 
 /* Test hook of the timeout path above. Arms the next attention launch of this cache
@@ -288,7 +291,8 @@ gca_status gca_set_wait_limit(gca_cache* cache, uint64_t wait_ns);
  * of its first key tile (nothing is ever in flight for that tile), so its MMA issuer's wait for
  * them runs out after the wait limit and the launch sets GCA_DEVERR_WAIT_TIMEOUT. The combine
  * launch of the call then does nothing (sticky error), so no output row that depends on a
- * split work unit is written; gca_check reports GCA_ERR_DEVICE until gca_reset. One-shot. */
+ * split work unit is written; gca_check reports GCA_ERR_DEVICE until gca_reset. One-shot; a call
+ * that takes the decode path (at most 4 query rows) clears it without effect. */
 gca_status gca_test_withhold_copies(gca_cache* cache);
 
 /* Fills *state from the host mirror (no GPU access). */
