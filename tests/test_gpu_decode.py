@@ -135,3 +135,29 @@ def test_sticky_error_makes_decode_a_noop():
     cache.attend(0, q_rot, out)
     torch.cuda.synchronize()
     assert bool((out == 3.0).all())
+
+
+def test_full_camera_stream_uses_eight_way_clusters():
+    # 1,024 frames with K = 1: ~80 key pages per head, so the decode launch splits every head
+    # over a full cluster of 8 CTAs
+    w = gi.workload("camera4").replace(permuted_free_list=True, seed=48)
+    cache = gca.GcaCache(gca.config_for(w), initial_free=gi.initial_free_list(w))
+    o = make_oracle(w)
+    ring = gi.draw_ring(w).cuda()
+    shape = (w.tokens_per_frame, w.num_heads, w.head_dim)
+    q_rot = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(q_rot)
+    for t in range(w.frames):
+        q, k, v = ring[t % w.ring]
+        cache.append_frame(t, q, k, v, q_rot)
+        o.append(t)
+        if t in (511, w.frames - 1):
+            cache.attend(t, q_rot, out)
+            torch.cuda.synchronize()
+            info = cache.attend_info()
+            assert info.launches == 1
+            if t == w.frames - 1:
+                assert info.grid == 8 * w.num_heads
+            check_book(cache, o.book, t)
+            check_attention(out.double().cpu().numpy(), o.attend(t), f"camera t={t}")
+    assert cache.check() == 0
