@@ -429,7 +429,30 @@ def run_stack(device, warm=1):
     e1.record(streams[0])
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
+    host_s = time.perf_counter() - t0
     assert all(c.check() == 0 for c in caches.values()), "device error in the stack"
+    # The same pass captured once as a CUDA graph (the four streams forked from and joined into
+    # the capturing one) and replayed: the device's own time, without the ~50,000 host calls.
+    graph = torch.cuda.CUDAGraph()
+    fork = torch.cuda.Event()
+    with torch.cuda.graph(graph, stream=streams[0]):
+        fork.record(streams[0])
+        for s in streams[1:]:
+            s.wait_event(fork)
+        one_pass(False)
+        for s in streams[1:]:
+            streams[0].wait_stream(s)
+    with torch.cuda.stream(streams[0]):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0.record(streams[0])
+    with torch.cuda.stream(streams[0]):
+        graph.replay()
+    e1.record(streams[0])
+    torch.cuda.synchronize()
+    g_ms = e0.elapsed_time(e1)
+    del graph
+    assert all(c.check() == 0 for c in caches.values()), "device error in the stack (graph)"
     layer_frames = w.frames * w.num_streams * w.num_layers
     for c in caches.values():
         c.close()
@@ -437,7 +460,10 @@ def run_stack(device, warm=1):
             "layer_frames_per_s": layer_frames / (ms / 1e3),
             "us_per_layer_frame": 1e3 * ms / layer_frames, "ms": ms,
             "attention_tflops_stream": flops[0] / (ms / 1e3) / 1e12,
-            "host_enqueue_s": round(time.perf_counter() - t0, 3)}
+            "host_enqueue_s": round(host_s, 3),
+            "graph_layer_frames_per_s": layer_frames / (g_ms / 1e3),
+            "graph_us_per_layer_frame": 1e3 * g_ms / layer_frames,
+            "graph_attention_tflops": flops[0] / (g_ms / 1e3) / 1e12}
 
 
 def run_configs(args, device, stream):
