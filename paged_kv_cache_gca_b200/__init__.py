@@ -28,6 +28,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 
 
 def library_path() -> str:
+    """The in-tree libgca.so built by paged_kv_cache_gca_b200.build, or the file GCA_LIBRARY
+    names (another build of this library, e.g. one compiled with different kernel settings)."""
     return os.environ.get("GCA_LIBRARY", os.path.join(_HERE, "libgca.so"))
 
 
