@@ -37,9 +37,61 @@ constexpr int kGroup = 4;  // pieces whose loads are issued together
 __device__ __forceinline__ void merge_row(const AttnParams& p, int u2, int qq, int h, int qi,
                                           int r, int col, int64_t c0, int64_t c1,
                                           unsigned int* wide) {
-  // Pieces are read in groups so that several loads are in flight per thread; they are summed
-  // in CTA order, as one at a time would.
   const int np = (int)(c1 - c0 + 1);
+  if (np <= kGroup) {
+    // the common case: every piece's (m, l) and O values in one round of loads, then the same
+    // arithmetic as below (maxima first, pieces summed in CTA order)
+    float2 ml[kGroup];
+    float4 v[kGroup][2];
+#pragma unroll
+    for (int k = 0; k < kGroup; ++k) {
+      if (k < np) {
+        const int64_t slot = part_slot(c0 + k, u2, qq);
+        ml[k] = __ldcg(&p.part_ml[slot * kTileQ + r]);
+        const float4* src =
+            reinterpret_cast<const float4*>(p.part_o + (slot * kTileQ + r) * kHeadDim + col);
+        v[k][0] = __ldcg(src);
+        v[k][1] = __ldcg(src + 1);
+      }
+    }
+    float M = -INFINITY, m_lo = INFINITY;
+#pragma unroll
+    for (int k = 0; k < kGroup; ++k) {
+      if (k < np) {
+        M = fmaxf(M, ml[k].x);
+        m_lo = fminf(m_lo, ml[k].x);
+      }
+    }
+    if (col == 0 && M - m_lo > 8.0f) atomicAdd_block(wide, 1u);
+    float acc[8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) acc[a] = 0.f;
+    float L = 0.f;
+#pragma unroll
+    for (int k = 0; k < kGroup; ++k) {
+      if (k >= np) break;
+      const float w = ex2(ml[k].x - M);
+      L += w * ml[k].y;
+      acc[0] += w * v[k][0].x;
+      acc[1] += w * v[k][0].y;
+      acc[2] += w * v[k][0].z;
+      acc[3] += w * v[k][0].w;
+      acc[4] += w * v[k][1].x;
+      acc[5] += w * v[k][1].y;
+      acc[6] += w * v[k][1].z;
+      acc[7] += w * v[k][1].w;
+    }
+    const float inv = 1.f / L;
+    uint4 o;
+    o.x = pack_bf2(acc[0] * inv, acc[1] * inv);
+    o.y = pack_bf2(acc[2] * inv, acc[3] * inv);
+    o.z = pack_bf2(acc[4] * inv, acc[5] * inv);
+    o.w = pack_bf2(acc[6] * inv, acc[7] * inv);
+    p.out[((int64_t)qi * p.H + h) * 8 + col / 8] = o;
+    return;
+  }
+  // More pieces: read in groups so that several loads are in flight per thread; they are summed
+  // in CTA order, as one at a time would.
   float M = -INFINITY, m_lo = INFINITY;
   for (int g = 0; g < np; g += kGroup) {
     float mx[kGroup];
