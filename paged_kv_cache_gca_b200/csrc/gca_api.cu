@@ -29,6 +29,13 @@ void nvtx_pop() { nvtxRangePop(); }
 namespace {
 
 constexpr int kMinStepsPerCta = 4;  // small launches (decode-like caches) spread wider
+// Planning cost of a CTA's move to another work unit, in key-tile steps (cta_begin): measured
+// per-CTA timelines put the move (epilogue, next Q tile, next first S) at ~4 us against ~1.1 us
+// per step. Applied while CTAs hold 16-128 steps on average: below, ranges are too short to
+// shift; above, the move is a small share of a CTA's time and the even split measured as fast.
+constexpr int kUnitGapSteps = 4;
+constexpr int kGapMinStepsPerCta = 16;
+constexpr int kGapMaxStepsPerCta = 128;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -205,14 +212,17 @@ bool plan_attention(const gca_cache* c, int64_t t, int64_t max_slots, AttnParams
   g = std::min<int64_t>(g, gmax);
   g = std::min<int64_t>(g, p->total);
   p->grid = (int32_t)g;
+  p->unit_gap = (p->total >= (int64_t)kGapMinStepsPerCta * g &&
+                 p->total <= (int64_t)kGapMaxStepsPerCta * g)
+                    ? kUnitGapSteps
+                    : 0;
   p->scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)cf.head_dim));
   p->wait_ns = c->wait_ns > 0 ? c->wait_ns : kDefaultWaitNs;
   p->withhold = c->withhold_next;
   bool sp = false;
   for (int u = 0; u < p->units2 && !sp; ++u) {
     const int64_t first = (int64_t)u * p->n_tiles;
-    sp = cta_of_step(first, p->total, p->grid) !=
-         cta_of_step(first + p->n_tiles - 1, p->total, p->grid);
+    sp = cta_of_step(first, *p) != cta_of_step(first + p->n_tiles - 1, *p);
   }
   *split = sp;
   *visible_keys = (na_frames + nwf) * L.T + c->traj_len;

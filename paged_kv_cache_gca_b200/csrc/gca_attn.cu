@@ -742,8 +742,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // A cache whose sticky error word is set gets no further work: every role sees an empty step
   // range and the CTA goes straight to its teardown.
   const bool dead = *reinterpret_cast<volatile uint32_t*>(p.err) != 0u;
-  const int64_t s_begin = (int64_t)blockIdx.x * p.total / p.grid;
-  const int64_t s_end = dead ? s_begin : (int64_t)(blockIdx.x + 1) * p.total / p.grid;
+  const int64_t s_begin = cta_begin(blockIdx.x, p);
+  const int64_t s_end = dead ? s_begin : cta_begin(blockIdx.x + 1, p);
 
   if (warp == kWarpTma) {
     tma_producer(&tm_k, &tm_v, p, sh, k_smem, v_smem, s_begin, s_end);

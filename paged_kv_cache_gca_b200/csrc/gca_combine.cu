@@ -149,7 +149,8 @@ __device__ __forceinline__ void merge_row(const AttnParams& p, int u2, int qq, i
 
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const AttnParams p) {
-  pdl_wait();  // the attention launch's partial records
+  // Which pieces hold this block's rows depends on the launch parameters alone: worked out
+  // before the wait, while the attention launch finishes.
   const int u = blockIdx.x / kBlocksPerTile;  // (head, query tile)
   const int r = (blockIdx.x % kBlocksPerTile) * kRowsPerBlock + threadIdx.x / kThreadsPerRow;
   const int col = (threadIdx.x % kThreadsPerRow) * 8;
@@ -158,9 +159,10 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const AttnPara
   const int u2 = h * p.n_pairs + qt / kQPerCta;
   const int qq = qt % kQPerCta;
   const int64_t first = (int64_t)u2 * p.n_tiles;
-  const int64_t c0 = cta_of_step(first, p.total, p.grid);
-  const int64_t c1 = cta_of_step(first + p.n_tiles - 1, p.total, p.grid);
-  if (c0 == c1) return;
+  const int64_t c0 = cta_of_step(first, p);
+  const int64_t c1 = cta_of_step(first + p.n_tiles - 1, p);
+  if (c0 == c1) return;  // not split: the attention kernel wrote these rows
+  pdl_wait();             // the attention launch's partial records
   const int qi = qt * kTileQ + r;
   __shared__ unsigned int wide;  // rows of this block merged over maxima > 2^8 apart
   __shared__ unsigned int dead;  // the cache's sticky error word (read once per block)

@@ -191,6 +191,7 @@ struct AttnParams {
   int32_t units2;        // H * n_pairs: work units of the attention kernel
   int64_t total;         // units2 * n_tiles
   int32_t grid;
+  int32_t unit_gap;      // planning cost of starting another work unit, in steps (cta_begin)
   float scale_log2;      // log2(e) / sqrt(D)
   uint64_t wait_ns;      // bound of every pipeline wait (a wait that runs out sets
                          // GCA_DEVERR_WAIT_TIMEOUT and the CTA winds down)
@@ -243,12 +244,32 @@ __device__ __forceinline__ void resolve_page(const AttnParams& p, int lp, int fa
   }
 }
 
-// Split bookkeeping shared by the attention and combine kernels: CTA c owns the flattened
-// (pair unit, key tile) steps [c*total/grid, (c+1)*total/grid); the CTA that holds step s is
-// ceil((s+1)*grid/total) - 1, and (CTA c, pair unit u2, query tile q of the pair) writes its
-// partial result to slot 2*(c + u2) + q. Over a launch the slots stay below 2*(grid + units2).
-__host__ __device__ inline int64_t cta_of_step(int64_t s, int64_t total, int64_t grid) {
-  return ((s + 1) * grid + total - 1) / total - 1;
+// Split bookkeeping shared by the host planner and the attention and combine kernels. The
+// flattened (pair unit, key tile) steps are cut into grid contiguous ranges of equal cost, where
+// a step costs 1 and every unit is followed by unit_gap more: a CTA that moves on to another
+// unit pays for that unit's start (its epilogue, the next Q tile, the next first S), so it gets
+// fewer steps. In cost coordinates unit u covers [u*span, u*span + n_tiles) with span = n_tiles
+// + unit_gap; CTA c starts at the step of cost c*units2*span/grid (a cut inside a gap moves to
+// the next unit's start). unit_gap = 0 is the even split [c*total/grid, (c+1)*total/grid).
+// (CTA c, pair unit u2, query tile q of the pair) writes its partial result to slot
+// 2*(c + u2) + q; ranges are monotone, so the slots of a launch are distinct and below
+// 2*(grid + units2).
+__host__ __device__ inline int64_t cta_begin(int64_t c, const AttnParams& p) {
+  const int64_t span = (int64_t)p.n_tiles + p.unit_gap;
+  const int64_t x = c * ((int64_t)p.units2 * span) / p.grid;
+  const int64_t u = x / span, off = x - u * span;
+  return u * p.n_tiles + (off < p.n_tiles ? off : (int64_t)p.n_tiles);
+}
+// The CTA whose range holds step s (0 <= s < total): the last c with cta_begin(c) <= s. Steps
+// never lie in a gap, so cta_begin(c) <= s exactly when c's cut X(c) = c*units2*span/grid is at
+// most the step's cost coordinate x = u*span + (s - u*n_tiles); the last such c is
+// ceil((x+1)*grid / (units2*span)) - 1 (an empty range is never returned).
+__host__ __device__ inline int64_t cta_of_step(int64_t s, const AttnParams& p) {
+  const int64_t span = (int64_t)p.n_tiles + p.unit_gap;
+  const int64_t u = s / p.n_tiles;
+  const int64_t x = u * span + (s - u * p.n_tiles);
+  const int64_t tc = (int64_t)p.units2 * span;
+  return ((x + 1) * p.grid + tc - 1) / tc - 1;
 }
 __host__ __device__ inline int64_t part_slot(int64_t cta, int64_t u2, int q) {
   return 2 * (cta + u2) + q;
