@@ -12,10 +12,11 @@
 // the two lanes of a key add their halves of q.k, the warp keeps an online softmax per query row
 // (row max in log2 units, row sum; lane l accumulates output dims 2l and 2l+1 from coalesced
 // 128-byte V rows, loaded together with the keys). Each CTA merges its warps with log-sum-exp
-// weights into shared memory; after a cluster barrier CTA 0 of the cluster reads the other
-// CTAs' results through distributed shared memory, merges them in rank order and writes the
-// output, and a second barrier keeps every CTA's shared memory alive until then. One launch,
-// no global scratch, and the result does not depend on CTA timing.
+// weights and stores the result into its own slot of CTA 0's shared memory (distributed shared
+// memory; a cluster barrier arrived at on entry and waited for before the stores makes sure CTA
+// 0 has started); after one cluster barrier CTA 0 merges the slots in rank order from its own
+// shared memory and writes the output. One launch, no global scratch, and the result does not
+// depend on CTA timing.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -61,13 +62,13 @@ __global__ void __launch_bounds__(32 * decode_warps<kRows>()) decode_kernel(cons
   __shared__ float sm_m[kDecodeWarps][kRows];
   __shared__ float sm_l[kDecodeWarps][kRows];
   __shared__ float sm_o[kDecodeWarps][kRows][kHeadDim];
-  __shared__ float cta_m[kRows], cta_l[kRows];  // this CTA's merged result, read by CTA 0
-  __shared__ float cta_o[kRows][kHeadDim];
-  __shared__ uint32_t dead;
-  if (threadIdx.x == 0) dead = *reinterpret_cast<volatile uint32_t*>(p.err);
-  __syncthreads();
-  // Sticky error: no output until gca_reset. Every CTA still passes both cluster barriers.
-  const bool live = dead == 0u;
+  // CTA 0's slots for every CTA's merged result (written remotely by each CTA)
+  __shared__ float cl_m[kDecodeMaxSplit][kRows], cl_l[kDecodeMaxSplit][kRows];
+  __shared__ float cl_o[kDecodeMaxSplit][kRows][kHeadDim];
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  // Sticky error: no output until gca_reset. Every CTA still takes part in the cluster
+  // barriers. The word, q and the first page ids are loaded together.
+  const bool live = *reinterpret_cast<volatile uint32_t*>(p.err) == 0u;
 
   // this lane's 32 dims of every query row, as bf16 pairs
   uint32_t qv[kRows][16];
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(32 * decode_warps<kRows>()) decode_kernel(cons
     const uint4* src = p.q + ((int64_t)r * p.H + h) * 8 + 4 * half;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const uint4 v = live ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 v = src[c];
       qv[r][4 * c + 0] = v.x;
       qv[r][4 * c + 1] = v.y;
       qv[r][4 * c + 2] = v.z;
@@ -94,10 +95,11 @@ __global__ void __launch_bounds__(32 * decode_warps<kRows>()) decode_kernel(cons
   }
 
   const int lp0 = (int)((int64_t)split * p.n_lp / n_split);
-  const int lp1 = live ? (int)((int64_t)(split + 1) * p.n_lp / n_split) : lp0;
+  const int lp1_all = (int)((int64_t)(split + 1) * p.n_lp / n_split);
   // the page id of the warp's next page is read while the current page is processed
   int next_page = 0, next_len = 0;
-  if (lp0 + warp < lp1) resolve_page(p, lp0 + warp, 0, &next_page, &next_len);
+  if (lp0 + warp < lp1_all) resolve_page(p, lp0 + warp, 0, &next_page, &next_len);
+  const int lp1 = live ? lp1_all : lp0;
   for (int lp = lp0 + warp; lp < lp1; lp += kDecodeWarps) {
     const int page = next_page, len = next_len;
     if (lp + kDecodeWarps < lp1) resolve_page(p, lp + kDecodeWarps, 0, &next_page, &next_len);
@@ -180,8 +182,8 @@ __global__ void __launch_bounds__(32 * decode_warps<kRows>()) decode_kernel(cons
   const int t_row = threadIdx.x / kHeadDim;  // row and dim this thread merges
   const int t_dim = threadIdx.x % kHeadDim;
   const bool merger = threadIdx.x < kRows * kHeadDim;
+  float M = -INFINITY, L = 0.f, O = 0.f;
   if (merger) {
-    float M = -INFINITY, L = 0.f, O = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, sm_m[w][t_row]);
 #pragma unroll
@@ -191,29 +193,32 @@ __global__ void __launch_bounds__(32 * decode_warps<kRows>()) decode_kernel(cons
       L = fmaf(wt, sm_l[w][t_row], L);
       O = fmaf(wt, sm_o[w][t_row][t_dim], O);
     }
-    cta_o[t_row][t_dim] = O;
+  }
+  // every CTA of the cluster has started (its arrival on entry), so CTA 0's shared memory
+  // exists: this CTA's result goes into its slot there
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  if (merger) {
+    *cluster.map_shared_rank(&cl_o[split][t_row][t_dim], 0) = O;
     if (t_dim == 0) {
-      cta_m[t_row] = M;
-      cta_l[t_row] = L;
+      *cluster.map_shared_rank(&cl_m[split][t_row], 0) = M;
+      *cluster.map_shared_rank(&cl_l[split][t_row], 0) = L;
     }
   }
-  // every CTA of the head has its result in shared memory
+  // every CTA's result is in CTA 0's shared memory (release / acquire)
   cluster.sync();
   if (split == 0 && merger && live) {
-    float M = -INFINITY;
-    for (int c = 0; c < n_split; ++c) M = fmaxf(M, *cluster.map_shared_rank(&cta_m[t_row], c));
-    float L = 0.f, O = 0.f;
+    float Mc = -INFINITY;
+    for (int c = 0; c < n_split; ++c) Mc = fmaxf(Mc, cl_m[c][t_row]);
+    float Lc = 0.f, Oc = 0.f;
     for (int c = 0; c < n_split; ++c) {
-      const float mc = *cluster.map_shared_rank(&cta_m[t_row], c);
-      const float wt = mc == -INFINITY ? 0.f : ex2(mc - M);  // splits without keys
-      L = fmaf(wt, *cluster.map_shared_rank(&cta_l[t_row], c), L);
-      O = fmaf(wt, *cluster.map_shared_rank(&cta_o[t_row][t_dim], c), O);
+      const float mc = cl_m[c][t_row];
+      const float wt = mc == -INFINITY ? 0.f : ex2(mc - Mc);  // splits without keys
+      Lc = fmaf(wt, cl_l[c][t_row], Lc);
+      Oc = fmaf(wt, cl_o[c][t_row][t_dim], Oc);
     }
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
-    out[((int64_t)t_row * p.H + h) * kHeadDim + t_dim] = __float2bfloat16_rn(O / L);
+    out[((int64_t)t_row * p.H + h) * kHeadDim + t_dim] = __float2bfloat16_rn(Oc / Lc);
   }
-  // CTA 0 has read every CTA's shared memory
-  cluster.sync();
   pdl_launch_dependents();
 }
 
