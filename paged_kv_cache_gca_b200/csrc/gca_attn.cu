@@ -15,9 +15,10 @@
 //
 // Work split: a CTA works on two 128-query tiles of one head at once (they see the same keys,
 // so every K/V tile is fetched once for both); a (head, tile pair) is a work unit. The flattened
-// (unit, key tile) steps are cut into `grid` equal ranges, one per CTA (one CTA per SM). A unit
-// that spans several CTAs leaves partial (O, row max, row sum) records per query tile that a
-// combine kernel merges with log-sum-exp weights.
+// (unit, key tile) steps are cut into `grid` contiguous ranges, one per CTA (one CTA per SM), of
+// equal cost: a CTA that moves on to another unit gets fewer key tiles (cta_begin). A unit that
+// spans several CTAs leaves partial (O, row max, row sum) records per query tile that a combine
+// kernel merges with log-sum-exp weights.
 //
 // CTA roles (352 threads):
 //   warps 0-3, 4-7  softmax warpgroup of query tile 0 / 1: thread r owns query row r (TMEM lane
